@@ -1,0 +1,135 @@
+"""Seeded synthetic inputs for the gen-tower attention layer.
+
+This module only draws random tensors; it holds none of the layer's arithmetic.
+It is the one piece shared by the CUDA path's callers (tests, bench) and the
+oracle's callers: both receive the very same bf16 tensors from here.
+
+Workload shapes follow the pages' workloads (DiffSynth-Studio "SenseNova-U1"
+page, quick-start and inference parameters: 2048x2048 default output, sides a
+multiple of 32; same page, architecture note: prompt encoded once into
+``past_key_values``; "Setup notes" page, "Why bf16 base on CPU + tower
+offload?": a static prefix-KV cache of a few hundred tokens per sample).
+Image tokens are 32-pixel patches, so 512^2 -> 256, 1024^2 -> 1024 and
+2048^2 -> 4096 tokens. Layer dimensions (hidden 4096, 32 query / 8 KV heads,
+head_dim 128) are those of the Qwen3-8B-class backbone the vLLM-Omni
+"SenseNova-U1" recipe names (Summary); the pages print no dims themselves.
+
+Distributions: hidden states, cached K/V and the upstream gradient N(0, 1);
+base weights N(0, 0.02); LoRA down (A) N(0, 1/16); LoRA up (B) N(0, 0.01);
+RMSNorm gains 1 + 0.1 N(0, 1). Each tensor is drawn in fp32 from its own CPU
+``torch.Generator`` seeded ``1000 * config + tensor_index`` and rounded to bf16.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import torch
+
+HIDDEN = 4096
+N_Q_HEADS = 32
+N_KV_HEADS = 8
+HEAD_DIM = 128
+RMS_EPS = 1e-6
+ROPE_THETA = 1e6
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerDims:
+    hidden: int = HIDDEN
+    n_q_heads: int = N_Q_HEADS
+    n_kv_heads: int = N_KV_HEADS
+    head_dim: int = HEAD_DIM
+    rms_eps: float = RMS_EPS
+    rope_theta: float = ROPE_THETA
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One layer call: B CFG branches of N image tokens over P cached keys."""
+    name: str
+    batch: int          # CFG branches (cond / uncond / image-uncond)
+    img_tokens: int     # N = (H/32) * (W/32)
+    prefix: int         # P = cached prefix keys per branch
+    lora_rank: int      # r (0 = no adapters)
+    lora_alpha: float
+    merged: bool = False   # LoRA folded into the base weights before the call
+    train: bool = False    # forward + LoRA backward
+    dims: LayerDims = LayerDims()
+
+
+# The five workloads: a 512^2 single-branch check, 1024^2 and 2048^2
+# text-to-image CFG (cond + fixed uncond), the 2048^2 dual-CFG edit with an
+# image prefix (400 text + 4096 image tokens) and merged LoRA, and the 2048^2
+# LoRA training step.
+WORKLOADS = {
+    0: Workload("fwd_512sq_b1", 1, 256, 64, 16, 16.0),
+    1: Workload("fwd_1024sq_cfg2", 2, 1024, 400, 32, 32.0),
+    2: Workload("fwd_2048sq_cfg2", 2, 4096, 400, 32, 32.0),
+    3: Workload("fwd_2048sq_edit_cfg3_merged", 3, 4096, 4496, 32, 32.0, merged=True),
+    4: Workload("train_2048sq_b1", 1, 4096, 400, 32, 32.0, train=True),
+}
+
+# tensor_index of each named tensor (seed = 1000 * config + tensor_index)
+_TENSOR_INDEX = {
+    "x": 0, "w_q": 1, "w_k": 2, "w_v": 3, "w_o": 4, "q_norm": 5, "k_norm": 6,
+    "a_q": 7, "a_k": 8, "a_v": 9, "a_o": 10, "b_q": 11, "b_k": 12, "b_v": 13,
+    "b_o": 14, "k_cache": 15, "v_cache": 16, "dy": 17,
+}
+
+
+def _draw(shape, std: float, mean: float, seed: int) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    t = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t.to(torch.bfloat16)
+
+
+def make_inputs(wl: Workload, seed_base: int, with_dy: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+    """Return CPU bf16 tensors for one layer call plus ``prefix_len`` (int32).
+
+    Shapes: x, dy [B, N, hidden]; w_q [Hq*dh, hidden]; w_k, w_v [Hkv*dh, hidden];
+    w_o [hidden, Hq*dh]; q_norm, k_norm [dh]; a_* [r, in]; b_* [out, r];
+    k_cache, v_cache [B, Hkv, P, dh] (keys already normalised and rotated).
+    """
+    d = wl.dims
+    B, N, P, r = wl.batch, wl.img_tokens, wl.prefix, wl.lora_rank
+    qd, kvd = d.n_q_heads * d.head_dim, d.n_kv_heads * d.head_dim
+    s = lambda name: seed_base + _TENSOR_INDEX[name]
+    out = {
+        "x": _draw((B, N, d.hidden), 1.0, 0.0, s("x")),
+        "w_q": _draw((qd, d.hidden), 0.02, 0.0, s("w_q")),
+        "w_k": _draw((kvd, d.hidden), 0.02, 0.0, s("w_k")),
+        "w_v": _draw((kvd, d.hidden), 0.02, 0.0, s("w_v")),
+        "w_o": _draw((d.hidden, qd), 0.02, 0.0, s("w_o")),
+        "q_norm": _draw((d.head_dim,), 0.1, 1.0, s("q_norm")),
+        "k_norm": _draw((d.head_dim,), 0.1, 1.0, s("k_norm")),
+        "k_cache": _draw((B, d.n_kv_heads, P, d.head_dim), 1.0, 0.0, s("k_cache")),
+        "v_cache": _draw((B, d.n_kv_heads, P, d.head_dim), 1.0, 0.0, s("v_cache")),
+    }
+    if r > 0:
+        for name, (rows, cols) in {
+            "a_q": (r, d.hidden), "a_k": (r, d.hidden), "a_v": (r, d.hidden), "a_o": (r, qd),
+            "b_q": (qd, r), "b_k": (kvd, r), "b_v": (kvd, r), "b_o": (d.hidden, r),
+        }.items():
+            std = 1.0 / 16.0 if name.startswith("a_") else 0.01
+            out[name] = _draw((rows, cols), std, 0.0, s(name))
+    if wl.train if with_dy is None else with_dy:
+        out["dy"] = _draw((B, N, d.hidden), 1.0, 0.0, s("dy"))
+    out["prefix_len"] = torch.full((B,), P, dtype=torch.int32)
+    return out
+
+
+def workload_inputs(index: int, with_dy: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+    return make_inputs(WORKLOADS[index], 1000 * index, with_dy)
+
+
+def tiny_workload(batch=2, img_tokens=5, prefix=3, lora_rank=2, lora_alpha=4.0, hidden=64,
+                  n_q_heads=4, n_kv_heads=2, head_dim=16, train=True) -> Workload:
+    """Small shapes for oracle checks (finite differences, brute force)."""
+    dims = LayerDims(hidden=hidden, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim)
+    return Workload("tiny", batch, img_tokens, prefix, lora_rank, lora_alpha, train=train, dims=dims)
