@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Throughput of the gen-tower attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one forward call of the layer (LoRA-down, QKV projection + LoRA up +
+QK-RMSNorm + RoPE, attention over [prefix cache ; self], LoRA-down o, O
+projection + LoRA up) on the 2048^2 text-to-image CFG workload: B = 2
+branches x N = 4096 image tokens (64 x 64 grid of 32-px patches), P = 400
+cached prefix keys, LoRA rank 32, hidden 4096, 32 / 8 heads, head_dim 128.
+Inputs are seeded synthetic tensors (mot_flow_matching_b200.synth), resident
+in HBM before timing; L2 is flushed (256 MiB write) before every timed step.
+Rank 0 prints one JSON line. Under torchrun every rank runs its own
+independent layer call (CFG branches / samples shard with no exchange), so
+scaling is weak and value = tokens of all ranks / max-over-ranks time.
+
+--impl reference times the CPU oracle (fp64 numpy) on the same workload, on a
+bounded sample of query rows per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gen-tower attn-layer image tokens/s at 1024²/2048²; % of BF16 tensor peak"
+UNIT = "image tokens/s"
+WORKLOAD_INDEX = 2          # 2048^2 text-to-image CFG layer call
+ALSO_INDEX = 1              # 1024^2 CFG, reported beside it
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def stage_work(wl, stage):
+    """Algorithmic (flops, bytes) of one launch of a stage."""
+    d = wl.dims
+    B, N, P, r = wl.batch, wl.img_tokens, wl.prefix, (0 if wl.merged else wl.lora_rank)
+    M, dh, Hq, Hkv, hid = B * N, d.head_dim, d.n_q_heads, d.n_kv_heads, d.hidden
+    qkv = (Hq + 2 * Hkv) * dh
+    L = P + N
+    if stage == "qkv_gemm":
+        return 2.0 * M * hid * qkv + 2.0 * M * r * qkv, 2.0 * (M * hid + qkv * hid + M * qkv)
+    if stage == "attn_fwd":
+        return 4.0 * B * Hq * N * L * dh, 2.0 * (B * Hq * N * dh + 2 * B * Hkv * L * dh + M * Hq * dh)
+    if stage == "o_gemm":
+        return 2.0 * M * Hq * dh * hid + 2.0 * M * r * hid, 2.0 * (M * Hq * dh + hid * Hq * dh + M * hid) + 4.0 * M * hid
+    if stage == "lora_down_qkv":
+        return 2.0 * M * hid * 3 * r, 2.0 * (M * hid + 3 * r * hid + M * 3 * r)
+    if stage == "lora_down_o":
+        return 2.0 * M * Hq * dh * r, 2.0 * (M * Hq * dh + r * Hq * dh + M * r)
+    if stage == "build_kv":
+        return 0.0, 2.0 * 2 * B * Hkv * P * dh * 2
+    if stage == "cvt_lora_o":
+        return 0.0, 2.0 * 2 * r * (Hq * dh + hid)
+    return 0.0, 0.0
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def oracle_sample(wl, inputs_cpu, rows_per_branch, seed=0):
+    """One oracle forward restricted to `rows_per_branch` query rows per branch."""
+    import numpy as np
+    from oracle import mot_attn_oracle as O
+    t64 = O.to_f64(inputs_cpu)
+    g = np.random.default_rng(seed)
+    rows = [np.sort(g.choice(wl.img_tokens, rows_per_branch, replace=False)) for _ in range(wl.batch)]
+    s = wl.lora_alpha / wl.lora_rank if wl.lora_rank else 0.0
+    t0 = time.perf_counter()
+    O.layer_forward(t64, O.dims_of(wl), s, query_rows=rows)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    from mot_flow_matching_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD_INDEX]
+    inputs = synth.workload_inputs(WORKLOAD_INDEX)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(wl, inputs, rows)
+    times = [oracle_sample(wl, inputs, rows, seed=i + 1) for i in range(args.steps)]
+    t = sum(times) / len(times)
+    value = wl.batch * rows / t
+    sample = (f"{rows} of {wl.img_tokens} query rows per branch, all {wl.img_tokens} keys/values projected, "
+              f"one oracle forward per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "img_tokens": wl.img_tokens, "prefix": wl.prefix,
+                   "lora_rank": wl.lora_rank, "parallelism": "none (CPU oracle, rank 0)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from mot_flow_matching_b200 import build as build_mod
+    from mot_flow_matching_b200 import synth
+    from mot_flow_matching_b200.layer import MotAttnLayer, mot_dev_profile, mot_dev_stage_times
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build_mod.build()
+    if world > 1:
+        dist.barrier()
+
+    def make(index):
+        wl = synth.WORKLOADS[index]
+        t = synth.workload_inputs(index)
+        td = {k: (v.to(dev) if k != "prefix_len" else v) for k, v in t.items()}
+        wts = {k: td[k] for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
+                                  "b_q", "b_k", "b_v", "b_o") if k in td}
+        layer = MotAttnLayer(wts, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_batch=wl.batch,
+                             max_img_tokens=wl.img_tokens, max_prefix=wl.prefix)
+        return wl, t, td, layer
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def device_steps(wl, td, layer, steps, warmup, profile):
+        x, kc, vc = td["x"], td["k_cache"], td["v_cache"]
+        pl = [int(v) for v in td["prefix_len"]]
+        y = torch.empty_like(x)
+        ws = layer.workspace(wl.batch, wl.img_tokens, wl.prefix, dev)
+        for _ in range(warmup):
+            layer.forward(x, kc, vc, pl, y=y, workspace=ws)
+        torch.cuda.synchronize(dev)
+        mot_dev_profile(layer.handle, profile)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        step_ms, stages = [], {}
+        launches = 0
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer.forward(x, kc, vc, pl, y=y, workspace=ws)
+            e1.record(stream)
+            launches += layer.last_launch_count()
+            e1.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+            if profile:
+                for name, ms in mot_dev_stage_times(layer.handle):
+                    stages.setdefault(name, []).append(ms)
+        torch.cuda.synchronize(dev)
+        mot_dev_profile(layer.handle, False)
+        return step_ms, stages, launches
+
+    wl, t_cpu, td, layer = make(WORKLOAD_INDEX)
+    clocks = ClockSampler(local)
+    clocks.start()
+    step_ms, stages, launches = device_steps(wl, td, layer, args.steps, args.warmup, True)
+    clk = clocks.stop()
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    tokens = wl.batch * wl.img_tokens
+    value = world * tokens * args.steps / (total_ms / 1e3)
+
+    # end to end through the public call with host buffers: pinned H2D of
+    # x and the prefix cache, the layer, D2H of y, every step
+    x_h = td["x"].cpu().pin_memory()
+    kc_h = td["k_cache"].cpu().pin_memory()
+    vc_h = td["v_cache"].cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    x_d, kc_d, vc_d = torch.empty_like(td["x"]), torch.empty_like(td["k_cache"]), torch.empty_like(td["v_cache"])
+    y_d = torch.empty_like(td["x"])
+    pl = [int(v) for v in td["prefix_len"]]
+    ws = layer.workspace(wl.batch, wl.img_tokens, wl.prefix, dev)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        kc_d.copy_(kc_h, non_blocking=True)
+        vc_d.copy_(vc_h, non_blocking=True)
+        layer.forward(x_d, kc_d, vc_d, pl, y=y_d, workspace=ws)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e2e_ms = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * tokens * args.steps / (e2e_ms / 1e3)
+    h2d = (x_h.numel() + kc_h.numel() + vc_h.numel()) * 2
+    d2h = y_h.numel() * 2
+
+    # 1024^2 CFG beside it (same protocol, fewer steps)
+    also = None
+    if not args.skip_also:
+        wl1, _, td1, layer1 = make(ALSO_INDEX)
+        ms1, _, _ = device_steps(wl1, td1, layer1, max(3, args.steps // 2), args.warmup, False)
+        also = {"workload": wl1.name, "value": wl1.batch * wl1.img_tokens / (statistics.mean(ms1) / 1e3),
+                "ms_per_step": statistics.mean(ms1)}
+        layer1.close()
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        total_flops = sum(stage_work(wl, s)[0] for s in stages)
+        stage_summary = {}
+        for name, v in stages.items():
+            fl, by = stage_work(wl, name)
+            avg = statistics.mean(v)
+            stage_summary[name] = {"ms": avg, "share": sum(v) / sum(sum(x) for x in stages.values()),
+                                   "tflops": fl / (avg / 1e3) / 1e12 if fl else None,
+                                   "gbs": by / (avg / 1e3) / 1e9}
+        top = max(stages, key=lambda n: sum(stages[n]))
+        fl, by = stage_work(wl, top)
+        avg_top = statistics.mean(stages[top])
+        if fl > 0:
+            achieved, peak, unit, bound = fl / (avg_top / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
+        else:
+            achieved, peak, unit, bound = by / (avg_top / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+        traffic = None
+        tf = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tf):
+            with open(tf) as f:
+                traffic = json.load(f).get(top)
+        cpu = None
+        if not args.no_cpu_baseline:
+            rows = args.cpu_rows
+            tcpu = oracle_sample(wl, t_cpu, rows)
+            cpu = {"value": wl.batch * rows / tcpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"one oracle forward over {rows} of {wl.img_tokens} query rows per branch "
+                             f"({wl.batch} branches; K/V of all tokens projected), {tcpu:.1f} s"}
+        layer_tflops = total_flops / (ms_per_step / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16+f16 (f32 accumulate)", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "img_tokens": wl.img_tokens,
+                       "prefix": wl.prefix, "lora_rank": wl.lora_rank, "hidden": wl.dims.hidden,
+                       "heads": [wl.dims.n_q_heads, wl.dims.n_kv_heads], "head_dim": wl.dims.head_dim,
+                       "parallelism": f"independent layer call per GPU x{world}",
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "layer_tflops": layer_tflops,
+            "pct_of_bf16_peak": 100.0 * layer_tflops / peaks["bf16_tflops"],
+            "roofline": {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} (burst)"},
+            "stages": stage_summary,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * world,
+            "clocks": clk,
+            "also": also,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-also", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

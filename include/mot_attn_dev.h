@@ -1,0 +1,57 @@
+/*
+ * mot_attn_dev.h -- kernel-level entry points of the same library, for tests
+ * that check one stage of the layer at a time. Same conventions as
+ * mot_attn.h (device/host pointers, 16-byte alignment, stream = cudaStream_t,
+ * host-side validation, no exceptions across the ABI).
+ */
+#ifndef MOT_ATTN_DEV_H
+#define MOT_ATTN_DEV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mot_attn.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* d = A B^T on the tensor cores (the persistent tcgen05 GEMM used by the
+ * layer's projections): a device [m, k], b device [n, k], both bf16
+ * (is_bf16 != 0) or both f16; d device f32 [m, n].
+ * Requires k % 64 == 0, n % 256 == 0, m >= 1. */
+mot_status mot_dev_gemm(const void* a, const void* b, float* d, int32_t m, int32_t n, int32_t k,
+                        int32_t is_bf16, void* stream);
+
+/* Byte offsets, inside the `saved` buffer of a training forward, of the
+ * activations it keeps (all device, f16 unless noted):
+ *   [0] q^      [B, Hq, N, dh]      normalised + rotated queries
+ *   [1] K       [B, Hkv, Lcap, dh]  keys: prefix rows then self rows
+ *   [2] V       [B, Hkv, Lcap, dh]
+ *   [3] o       [B*N, Hq*dh]        attention output (o_proj input)
+ *   [4] lse     f32 [B, Hq, N]      natural-log softmax normaliser
+ *   [5] xhat    [B*N, (Hq+Hkv)*dh]  normalised pre-gain q/k
+ *   [6] rstd    f32 [B*N, Hq+Hkv]
+ *   [7] u_qkv   bf16 [B*N, 3*RP]    s x A^T per q/k/v (RP = rank rounded up to 64)
+ *   [8] u_o     [B*N, RP]           s o A_o^T
+ * lcap receives Lcap = round_up(P_max + N, 128). */
+mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32_t img_tokens,
+                                int32_t prefix_max, size_t offsets[9], int32_t* lcap);
+
+/* Per-stage device timing. enable != 0: every later forward/backward call
+ * records a CUDA event on its stream before its first launch and after each
+ * launch (no synchronisation is added). mot_dev_stage_times waits for the
+ * last call's final event and writes, for each launch of that call in order,
+ * its stage id and its duration in milliseconds (at most `max` entries;
+ * *count receives the number of launches). */
+mot_status mot_dev_profile(mot_attn_t h, int32_t enable);
+mot_status mot_dev_stage_times(mot_attn_t h, int32_t* ids, float* ms, int32_t max, int32_t* count);
+
+/* Static name of a stage id ("qkv_gemm", "attn_fwd", ...; "?" if unknown). */
+const char* mot_dev_stage_name(int32_t id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOT_ATTN_DEV_H */

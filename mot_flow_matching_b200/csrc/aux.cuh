@@ -1,0 +1,118 @@
+// aux.cuh -- bandwidth-bound helper kernels (no tensor cores).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace mot {
+
+struct PlenArray {
+  int v[kMaxBatch];
+};
+
+// Build the attention key/value buffers [B, Hkv, Lcap, dh] (f16) around the
+// self rows the QKV epilogue writes: rows [0, plen[b]) take the cached prefix
+// (bf16 -> f16, exact for |x| <= 65504 apart from f16 subnormals), rows
+// [plen[b] + N, Lcap) are zeroed so masked key tiles never hold NaN/Inf.
+// "Setup notes" (LoRA trainer docs): the prefix-KV cache is static input.
+// One thread moves 8 elements (16 bytes).
+__global__ void __launch_bounds__(256) build_kv_kernel(const __nv_bfloat16* __restrict__ kc,
+                                                       const __nv_bfloat16* __restrict__ vc,
+                                                       __half* __restrict__ kall, __half* __restrict__ vall,
+                                                       int Hkv, int Pmax, int N, int Lcap, long long total_chunks,
+                                                       PlenArray plen, int* status) {
+  bool overflow = false;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total_chunks;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int chunk = static_cast<int>(idx & 15);
+    const long long rowg = idx >> 4;
+    const int row = static_cast<int>(rowg % Lcap);
+    const long long bg = rowg / Lcap;
+    const int b = static_cast<int>(bg / Hkv);
+    const int pl = plen.v[b];
+    uint4* kd = reinterpret_cast<uint4*>(kall + rowg * 128 + chunk * 8);
+    uint4* vd = reinterpret_cast<uint4*>(vall + rowg * 128 + chunk * 8);
+    if (row < pl) {
+      const long long src = (bg * Pmax + row) * 128 + chunk * 8;
+      const uint4 kr = *reinterpret_cast<const uint4*>(kc + src);
+      const uint4 vr = *reinterpret_cast<const uint4*>(vc + src);
+      const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kr);
+      const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&vr);
+      uint4 ko, vo;
+      uint32_t* ko32 = reinterpret_cast<uint32_t*>(&ko);
+      uint32_t* vo32 = reinterpret_cast<uint32_t*>(&vo);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float k0 = __bfloat162float(kb[2 * i]), k1 = __bfloat162float(kb[2 * i + 1]);
+        const float v0 = __bfloat162float(vb[2 * i]), v1 = __bfloat162float(vb[2 * i + 1]);
+        overflow |= fabsf(k0) > 65504.f || fabsf(k1) > 65504.f || fabsf(v0) > 65504.f || fabsf(v1) > 65504.f;
+        ko32[i] = pack_half2(k0, k1);
+        vo32[i] = pack_half2(v0, v1);
+      }
+      *kd = ko;
+      *vd = vo;
+    } else if (row >= pl + N) {
+      *kd = make_uint4(0, 0, 0, 0);
+      *vd = make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
+}
+
+// dst[i] = f16(src[i]) for n elements (n % 8 == 0, 16-byte aligned).
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src,
+                                                          __half* __restrict__ dst, long long n8, int* status) {
+  bool overflow = false;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 r = reinterpret_cast<const uint4*>(src)[i];
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&r);
+    uint4 o;
+    uint32_t* o32 = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = __bfloat162float(bv[2 * k]), b = __bfloat162float(bv[2 * k + 1]);
+      overflow |= fabsf(a) > 65504.f || fabsf(b) > 65504.f;
+      o32[k] = pack_half2(a, b);
+    }
+    reinterpret_cast<uint4*>(dst)[i] = o;
+  }
+  if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
+}
+
+// LoRA bake-in ("SenseNova-U1.5" vLLM-Omni recipe, 8-step distilled LoRA:
+// fused into the gen tower at load):
+//   out[i, j] = RNE_bf16(w[i, j] + s * sum_k b[i, k] a[k, j]),
+// the sum over k ascending in f32, then one f32 fma and one rounding to bf16.
+// out may alias w (each element reads its own w before writing it).
+// Block: 32 x 8 threads over a 8-row x 256-column patch; b rows staged in smem.
+__global__ void __launch_bounds__(256) merge_lora_kernel(const __nv_bfloat16* w, const __nv_bfloat16* __restrict__ a,
+                                                         const __nv_bfloat16* __restrict__ bm, __nv_bfloat16* out,
+                                                         int rows, int cols, int r, float s) {
+  __shared__ float sb[8][128];
+  const int i0 = blockIdx.y * 8;
+  for (int t = threadIdx.y * 32 + threadIdx.x; t < 8 * r; t += 256) {
+    const int ii = t / r, k = t % r;
+    sb[ii][k] = (i0 + ii < rows) ? __bfloat162float(bm[static_cast<long long>(i0 + ii) * r + k]) : 0.f;
+  }
+  __syncthreads();
+  const int i = i0 + threadIdx.y;
+  if (i >= rows) return;
+#pragma unroll 1
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = blockIdx.x * 256 + jj * 32 + threadIdx.x;
+    if (j >= cols) break;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < r; ++k) acc = fmaf(sb[threadIdx.y][k], __bfloat162float(a[static_cast<long long>(k) * cols + j]), acc);
+    const long long o = static_cast<long long>(i) * cols + j;
+    out[o] = __float2bfloat16_rn(fmaf(s, acc, __bfloat162float(w[o])));
+  }
+}
+
+// f32 copy of a bf16 vector (norm gains)
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = __bfloat162float(src[i]);
+}
+
+}  // namespace mot

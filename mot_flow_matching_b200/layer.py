@@ -1,0 +1,195 @@
+"""Python binding of the C ABI: argument marshalling only.
+
+The module-level functions carry the C names (``mot_attn_create``,
+``mot_attn_forward``, ...) and take torch tensors where the C call takes
+device pointers; every step of the layer runs in libmotattn.so.
+``MotAttnLayer`` bundles a handle with the buffers a caller needs.
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import byref, c_int32, c_size_t, c_void_p
+from typing import Dict, Optional, Sequence, Tuple
+
+import torch
+
+from ._abi import MotAttnConfig, MotAttnWeights, check, lib
+
+WEIGHT_NAMES = ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
+                "b_q", "b_k", "b_v", "b_o")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmotattn must be contiguous")
+    return c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def make_config(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, lora_rank=0, lora_alpha=0.0,
+                rms_eps=1e-6, rope_theta=1e6, max_batch=1, max_img_tokens=256, max_prefix=0,
+                enable_backward=False) -> MotAttnConfig:
+    return MotAttnConfig(hidden, n_q_heads, n_kv_heads, head_dim, lora_rank, float(lora_alpha), float(rms_eps),
+                         float(rope_theta), max_batch, max_img_tokens, max_prefix, int(bool(enable_backward)))
+
+
+def mot_attn_query_sizes(cfg: MotAttnConfig, batch: int, img_tokens: int, prefix_max: int) -> Tuple[int, int]:
+    ws, sv = c_size_t(0), c_size_t(0)
+    check(lib().mot_attn_query_sizes(byref(cfg), batch, img_tokens, prefix_max, byref(ws), byref(sv)),
+          "mot_attn_query_sizes")
+    return ws.value, sv.value
+
+
+def mot_attn_create(cfg: MotAttnConfig, weights: Dict[str, torch.Tensor], stream=None) -> c_void_p:
+    w = MotAttnWeights(*[_ptr(weights.get(n)) for n in WEIGHT_NAMES])
+    h = c_void_p()
+    check(lib().mot_attn_create(byref(cfg), byref(w), _stream(stream), byref(h)), "mot_attn_create")
+    return h
+
+
+def mot_attn_forward(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max, y,
+                     y_f32=None, saved=None, workspace=None, stream=None) -> None:
+    pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
+    check(lib().mot_attn_forward(h, _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl, prefix_max,
+                                 _ptr(y), _ptr(y_f32), _ptr(saved), saved.numel() if saved is not None else 0,
+                                 _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                 _stream(stream)), "mot_attn_forward")
+
+
+def mot_attn_backward(h, dy, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max,
+                      saved, dx, dx_f32=None, d_a=None, d_b=None, accumulate=False, workspace=None,
+                      stream=None) -> None:
+    pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
+    da = (c_void_p * 4)(*[_ptr(t) for t in (d_a or [None] * 4)])
+    db = (c_void_p * 4)(*[_ptr(t) for t in (d_b or [None] * 4)])
+    check(lib().mot_attn_backward(h, _ptr(dy), _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl,
+                                  prefix_max, _ptr(saved), saved.numel() if saved is not None else 0, _ptr(dx),
+                                  _ptr(dx_f32), da, db, int(bool(accumulate)), _ptr(workspace),
+                                  workspace.numel() if workspace is not None else 0, _stream(stream)),
+          "mot_attn_backward")
+
+
+def mot_attn_merge_lora(h, w_q_out, w_k_out, w_v_out, w_o_out, stream=None) -> None:
+    check(lib().mot_attn_merge_lora(h, _ptr(w_q_out), _ptr(w_k_out), _ptr(w_v_out), _ptr(w_o_out),
+                                    _stream(stream)), "mot_attn_merge_lora")
+
+
+def mot_attn_get_device_status(h, stream=None) -> int:
+    return lib().mot_attn_get_device_status(h, _stream(stream))
+
+
+def mot_attn_destroy(h) -> None:
+    lib().mot_attn_destroy(h)
+
+
+def mot_attn_last_launch_count(h) -> int:
+    return lib().mot_attn_last_launch_count(h)
+
+
+def mot_status_string(status: int) -> str:
+    return lib().mot_status_string(status).decode()
+
+
+def mot_dev_gemm(a, b, d, stream=None) -> None:
+    m, k = a.shape
+    n = b.shape[0]
+    check(lib().mot_dev_gemm(_ptr(a), _ptr(b), _ptr(d), m, n, k, int(a.dtype == torch.bfloat16),
+                             _stream(stream)), "mot_dev_gemm")
+
+
+def mot_dev_saved_layout(cfg: MotAttnConfig, batch, img_tokens, prefix_max):
+    offs = (c_size_t * 9)()
+    lcap = c_int32(0)
+    check(lib().mot_dev_saved_layout(byref(cfg), batch, img_tokens, prefix_max, offs, byref(lcap)),
+          "mot_dev_saved_layout")
+    return list(offs), lcap.value
+
+
+def mot_dev_profile(h, enable: bool) -> None:
+    check(lib().mot_dev_profile(h, int(bool(enable))), "mot_dev_profile")
+
+
+def mot_dev_stage_times(h, max_stages: int = 32):
+    ids = (c_int32 * max_stages)()
+    ms = (ctypes.c_float * max_stages)()
+    count = c_int32(0)
+    check(lib().mot_dev_stage_times(h, ids, ms, max_stages, byref(count)), "mot_dev_stage_times")
+    return [(lib().mot_dev_stage_name(ids[i]).decode(), ms[i]) for i in range(min(count.value, max_stages))]
+
+
+class MotAttnLayer:
+    """A handle plus the caller-owned buffers of one call shape."""
+
+    def __init__(self, weights: Dict[str, torch.Tensor], lora_rank: int = 0, lora_alpha: float = 0.0,
+                 max_batch: int = 1, max_img_tokens: int = 256, max_prefix: int = 0,
+                 enable_backward: bool = False, hidden: int = 4096, n_q_heads: int = 32, n_kv_heads: int = 8,
+                 head_dim: int = 128, rms_eps: float = 1e-6, rope_theta: float = 1e6, stream=None):
+        self.cfg = make_config(hidden, n_q_heads, n_kv_heads, head_dim, lora_rank, lora_alpha, rms_eps,
+                               rope_theta, max_batch, max_img_tokens, max_prefix, enable_backward)
+        self.weights = dict(weights)  # keep the tensors alive
+        self.handle = mot_attn_create(self.cfg, self.weights, stream)
+        self._ws = None
+
+    def sizes(self, batch, img_tokens, prefix_max):
+        return mot_attn_query_sizes(self.cfg, batch, img_tokens, prefix_max)
+
+    def workspace(self, batch, img_tokens, prefix_max, device="cuda"):
+        ws, _ = self.sizes(batch, img_tokens, prefix_max)
+        if self._ws is None or self._ws.numel() < ws:
+            self._ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def new_saved(self, batch, img_tokens, prefix_max, device="cuda"):
+        _, sv = self.sizes(batch, img_tokens, prefix_max)
+        return torch.empty(sv, dtype=torch.uint8, device=device)
+
+    def forward(self, x, k_cache, v_cache, prefix_len, y=None, y_f32=None, saved=None, workspace=None,
+                stream=None):
+        B, N, d = x.shape
+        P = k_cache.shape[2] if k_cache is not None else 0
+        if y is None:
+            y = torch.empty_like(x)
+        if workspace is None:
+            workspace = self.workspace(B, N, P, x.device)
+        mot_attn_forward(self.handle, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, saved, workspace, stream)
+        return y
+
+    def backward(self, dy, x, k_cache, v_cache, prefix_len, saved, dx=None, dx_f32=None, d_a=None, d_b=None,
+                 accumulate=False, workspace=None, stream=None):
+        B, N, d = x.shape
+        P = k_cache.shape[2] if k_cache is not None else 0
+        if dx is None:
+            dx = torch.empty_like(x)
+        if workspace is None:
+            workspace = self.workspace(B, N, P, x.device)
+        mot_attn_backward(self.handle, dy, x, B, N, k_cache, v_cache, prefix_len, P, saved, dx, dx_f32, d_a, d_b,
+                          accumulate, workspace, stream)
+        return dx
+
+    def merge_lora(self, w_q_out, w_k_out, w_v_out, w_o_out, stream=None):
+        mot_attn_merge_lora(self.handle, w_q_out, w_k_out, w_v_out, w_o_out, stream)
+        self.weights.update(w_q=w_q_out, w_k=w_k_out, w_v=w_v_out, w_o=w_o_out)
+
+    def device_status(self, stream=None) -> int:
+        return mot_attn_get_device_status(self.handle, stream)
+
+    def last_launch_count(self) -> int:
+        return mot_attn_last_launch_count(self.handle)
+
+    def close(self):
+        if self.handle is not None:
+            mot_attn_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
