@@ -23,9 +23,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +34,27 @@ UNIT = "image tokens/s"
 WORKLOAD_INDEX = 2          # 2048^2 text-to-image CFG layer call
 ALSO_INDEX = 1              # 1024^2 CFG, reported beside it
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the 2048^2 CFG workload, keyed by the sha256 of the
+# kernel's source file at capture time: a changed kernel reports null.
+TRAFFIC = {
+    "attn_fwd": {"sha256": "6877987e024f348e6437d4696ef38d21d6ecef3ec714f3f9e9f46d781518cf00",
+                 "bytes": 104920576 + 34853632},
+}
+KERNEL_SOURCES = {"attn_fwd": "attn_fwd.cuh", "qkv_gemm": "gemm.cuh", "o_gemm": "gemm.cuh"}
+
+
+def kernel_traffic(stage):
+    import hashlib
+    src = KERNEL_SOURCES.get(stage)
+    entry = TRAFFIC.get(stage)
+    if not src or not entry:
+        return None
+    path = os.path.join(ROOT, "mot_flow_matching_b200", "csrc", src)
+    with open(path, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return entry["bytes"] if sha == entry["sha256"] else None
 
 
 def load_peaks():
@@ -72,50 +91,59 @@ def stage_work(wl, stage):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock and throttle reasons of this process's GPU, sampled every
+    10 ms through NVML from a background thread while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self, nvml):
+        import torch
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return nvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nvml.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml as nvml
+            nvml.nvmlInit()
+            h = self._handle(nvml)
+            self.max_mhz = float(nvml.nvmlDeviceGetMaxClockInfo(h, nvml.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report that, do not guess
+            self.reasons.add(f"nvml unavailable: {type(e).__name__}")
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM)))
+                    bits = nvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for bit, name in self.REASONS.items():
+                        if bits & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                self._stop.wait(0.01)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def dist_setup():
@@ -174,6 +202,30 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_once(args):
+    """One warm forward of a workload (the target of ncu captures)."""
+    import torch
+    from mot_flow_matching_b200 import build as build_mod
+    from mot_flow_matching_b200 import synth
+    from mot_flow_matching_b200.layer import MotAttnLayer
+    build_mod.build()
+    wl = synth.WORKLOADS[args.workload]
+    t = synth.workload_inputs(args.workload)
+    td = {k: (v.cuda() if k != "prefix_len" else v) for k, v in t.items()}
+    wts = {k: td[k] for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
+                              "b_q", "b_k", "b_v", "b_o") if k in td}
+    layer = MotAttnLayer(wts, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_batch=wl.batch,
+                         max_img_tokens=wl.img_tokens, max_prefix=wl.prefix)
+    pl = [int(v) for v in td["prefix_len"]]
+    for _ in range(2):
+        y = layer.forward(td["x"], td["k_cache"], td["v_cache"], pl)
+    torch.cuda.synchronize()
+    status = layer.device_status()
+    layer.close()
+    print(json.dumps({"once": wl.name, "status": status, "y_abs_mean": float(y.float().abs().mean())}))
+    return 0 if status == 0 else 1
 
 
 def run_ours(args):
@@ -319,11 +371,7 @@ def run_ours(args):
             achieved, peak, unit, bound = fl / (avg_top / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
         else:
             achieved, peak, unit, bound = by / (avg_top / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
-        traffic = None
-        tf = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(tf):
-            with open(tf) as f:
-                traffic = json.load(f).get(top)
+        traffic = kernel_traffic(top)
         cpu = None
         if not args.no_cpu_baseline:
             rows = args.cpu_rows
@@ -371,7 +419,11 @@ def main():
     ap.add_argument("--skip-also", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--once", action="store_true", help="one warm forward, no timing (ncu target)")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX)
     args = ap.parse_args()
+    if args.once:
+        return run_once(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
