@@ -161,6 +161,28 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
 mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void* w_v_out,
                                void* w_o_out, void* stream);
 
+/* Forward that allocates nothing and takes no workspace. The pages describe
+ * no such call; it exists for callers that cannot call cudaMalloc per call:
+ * plug-ins whose host owns all device memory (pre-reserved arenas where an
+ * extra allocation fails or fragments the pool) and latency-critical loops
+ * where cudaMalloc's implicit device-wide synchronisation is not acceptable.
+ * Arguments are those of mot_attn_forward without saved/workspace
+ * (inference only). The scratch lives in one 32 MiB device array inside this
+ * library (every GPU that loads the library holds it until process exit);
+ * a call whose scratch exceeds 32 MiB returns MOT_ERR_WORKSPACE_TOO_SMALL
+ * before anything is enqueued (at hidden 4096, LoRA rank 32 and a 400-token
+ * prefix that is about 1400 image tokens in one branch; the workspace_bytes
+ * of mot_attn_query_sizes is the exact need).
+ * The first call on a device resolves the array's device address on the
+ * host; make that first call before any stream capture. All calls share the
+ * one array and leave their intermediates in it: calls that overlap on the
+ * GPU (other streams, other handles, other threads) race and must be
+ * serialised by the caller. Nothing in the array needs to start at zero:
+ * every byte a call reads was written earlier in the same call. */
+mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int32_t batch, int32_t img_tokens,
+                                    const void* k_cache, const void* v_cache, const int32_t* prefix_len,
+                                    int32_t prefix_max, void* y, float* y_f32, void* stream);
+
 /* Synchronise `stream` and return (and clear) the status latched on the
  * device by earlier calls: MOT_OK, MOT_ERR_NUMERIC or MOT_ERR_TIMEOUT. */
 mot_status mot_attn_get_device_status(mot_attn_t h, void* stream);

@@ -47,6 +47,8 @@ SIGNATURES = {
     "mot_attn_backward": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                     POINTER(c_int32), c_int32, c_void_p, c_size_t, c_void_p, c_void_p,
                                     POINTER(c_void_p), POINTER(c_void_p), c_int32, c_void_p, c_size_t, c_void_p]),
+    "mot_attn_forward_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
+                                           POINTER(c_int32), c_int32, c_void_p, c_void_p, c_void_p]),
     "mot_attn_merge_lora": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "mot_attn_get_device_status": (c_int32, [c_void_p, c_void_p]),
     "mot_attn_destroy": (None, [c_void_p]),

@@ -593,6 +593,50 @@ mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void*
   return build_weight_maps(h);
 }
 
+// ------------------------------------------------------------------ no-allocation forward
+// Scratch of mot_attn_forward_noalloc: one file-scope device array. In host
+// code `g_noalloc_scratch` names a host-side stand-in, not device memory, so
+// its device address is looked up with cudaGetSymbolAddress once per device
+// (with that device current) and only that address is handed to kernels.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (resolved on the
+// first call per device); nullptr on failure.
+void* noalloc_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int32_t B, int32_t N,
+                                               const void* k_cache, const void* v_cache,
+                                               const int32_t* prefix_len, int32_t P, void* y, float* y_f32,
+                                               void* stream) {
+  if (!h || !x || !y || !prefix_len) return MOT_ERR_INVALID_ARGUMENT;
+  if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
+  size_t need = 0;
+  const mot_status st = mot_attn_query_sizes(&h->cfg, B, N, P, &need, nullptr);
+  if (st != MOT_OK) return st;
+  if (need > kNoAllocScratchBytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return MOT_ERR_CUDA;
+  return mot_attn_forward(h, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, nullptr, 0, scratch,
+                          kNoAllocScratchBytes, stream);
+}
+
 // ------------------------------------------------------------------ dev entry points
 mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, int32_t n, int32_t k, int32_t is_bf16,
                         void* stream) {

@@ -63,6 +63,16 @@ def mot_attn_forward(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequ
                                  _stream(stream)), "mot_attn_forward")
 
 
+def mot_attn_forward_noalloc(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max,
+                             y, y_f32=None, stream=None) -> None:
+    """Forward whose scratch is the library's own fixed device array (no
+    workspace argument, no allocation); see include/mot_attn.h."""
+    pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
+    check(lib().mot_attn_forward_noalloc(h, _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl,
+                                         prefix_max, _ptr(y), _ptr(y_f32), _stream(stream)),
+          "mot_attn_forward_noalloc")
+
+
 def mot_attn_backward(h, dy, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max,
                       saved, dx, dx_f32=None, d_a=None, d_b=None, accumulate=False, workspace=None,
                       stream=None) -> None:
