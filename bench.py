@@ -86,7 +86,26 @@ def stage_work(wl, stage):
     if stage == "build_kv":
         return 0.0, 2.0 * 2 * B * Hkv * P * dh * 2
     if stage == "cvt_lora_o":
-        return 0.0, 2.0 * 2 * r * (Hq * dh + hid)
+        return 0.0, 2.0 * 2 * r * (Hq * dh + hid + qkv)
+    # backward (LoRA training): base, gains and cache frozen
+    if stage == "bwd_do_gemm":
+        return 2.0 * M * hid * Hq * dh + 2.0 * M * r * Hq * dh, 2.0 * (M * hid + hid * Hq * dh + 2 * M * Hq * dh)
+    if stage in ("bwd_g_o", "bwd_db_o"):
+        return 2.0 * M * hid * r, 2.0 * (M * hid + M * r)
+    if stage == "bwd_da_o":
+        return 2.0 * M * Hq * dh * r, 2.0 * (M * Hq * dh + M * r)
+    if stage == "attn_bwd_dq":   # S, dP and dQ over all L keys
+        return 6.0 * B * Hq * N * L * dh, 2.0 * (2 * B * Hq * N * dh + 2 * B * Hkv * L * dh + M * qkv)
+    if stage == "attn_bwd_dkv":  # dK and dV over the N self keys (S, dP recomputed on top)
+        return 4.0 * B * Hq * N * N * dh, 2.0 * (2 * B * Hq * N * dh + 2 * B * Hkv * N * dh)
+    if stage in ("bwd_g_qkv", "bwd_db_qkv"):
+        return 2.0 * M * qkv * r / 3.0, 2.0 * (M * qkv + M * r) / 3.0
+    if stage == "bwd_da_qkv":
+        return 2.0 * M * hid * r, 2.0 * (M * hid + M * r)
+    if stage == "bwd_dx_gemm":
+        return 2.0 * M * qkv * hid + 2.0 * M * 3 * r * hid, 2.0 * (M * qkv + qkv * hid + M * hid) + 4.0 * M * hid
+    if stage == "bwd_cvt_lora":
+        return 0.0, 2.0 * 2 * r * qkv
     return 0.0, 0.0
 
 
@@ -228,6 +247,74 @@ def run_once(args):
     return 0 if status == 0 else 1
 
 
+TRAIN_INDEX = 4  # 2048^2 LoRA training layer call: B = 1, N = 4096, P = 400, r = 32
+
+
+def train_steps(bundle, dev, flush, stream, args, world):
+    """Forward (activations kept) + backward of the training workload; each
+    timed separately with CUDA events, per-launch times from the library."""
+    import torch
+    import torch.distributed as dist
+    from mot_flow_matching_b200.layer import mot_dev_profile, mot_dev_stage_times
+    wl, td, layer = bundle
+    pl = [int(v) for v in td["prefix_len"]]
+    x, kc, vc, dy = td["x"], td["k_cache"], td["v_cache"], td["dy"]
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    sv = layer.new_saved(wl.batch, wl.img_tokens, wl.prefix, dev)
+    ws = layer.workspace(wl.batch, wl.img_tokens, wl.prefix, dev)
+    names = ("q", "k", "v", "o")
+    d_a = [torch.zeros(td["a_" + n].shape, device=dev) for n in names]
+    d_b = [torch.zeros(td["b_" + n].shape, device=dev) for n in names]
+
+    def step():
+        layer.forward(x, kc, vc, pl, y=y, saved=sv, workspace=ws)
+        layer.backward(dy, x, kc, vc, pl, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    mot_dev_profile(layer.handle, True)
+    fwd_ms, bwd_ms, stages, launches = [], [], {}, 0
+    for _ in range(args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        layer.forward(x, kc, vc, pl, y=y, saved=sv, workspace=ws)
+        e[1].record(stream)
+        launches += layer.last_launch_count()
+        for name, ms in mot_dev_stage_times(layer.handle):
+            stages.setdefault(name, []).append(ms)
+        layer.backward(dy, x, kc, vc, pl, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
+        e[2].record(stream)
+        launches += layer.last_launch_count()
+        e[2].synchronize()
+        for name, ms in mot_dev_stage_times(layer.handle):
+            stages.setdefault(name, []).append(ms)
+        fwd_ms.append(e[0].elapsed_time(e[1]))
+        bwd_ms.append(e[1].elapsed_time(e[2]))
+    mot_dev_profile(layer.handle, False)
+    assert layer.device_status() == 0
+    layer.close()
+    f, b = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    fwd_flops = sum(stage_work(wl, n)[0] for n in ("lora_down_qkv", "qkv_gemm", "attn_fwd", "lora_down_o", "o_gemm"))
+    bwd_flops = sum(stage_work(wl, n)[0] * (3 if n in ("bwd_g_qkv", "bwd_db_qkv", "bwd_da_qkv") else 1)
+                    for n in stages if n.startswith(("bwd_", "attn_bwd")))
+    peaks, _ = load_peaks()
+    per = {}
+    for n, v in stages.items():
+        mult = 3 if n in ("bwd_g_qkv", "bwd_db_qkv", "bwd_da_qkv") else 1
+        ms = sum(v) / args.steps  # per step (the q/k/v stages launch three times)
+        fl = stage_work(wl, n)[0] * mult
+        per[n] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12 if fl else None}
+    return {"workload": wl.name, "fwd_ms": f, "bwd_ms": b, "tokens_per_s": world * wl.batch * wl.img_tokens / ((f + b) / 1e3),
+            "fwd_tflops": fwd_flops / (f / 1e3) / 1e12, "bwd_tflops": bwd_flops / (b / 1e3) / 1e12,
+            "bwd_pct_of_bf16_peak": 100.0 * bwd_flops / (b / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "bwd_algorithmic_gflop": bwd_flops / 1e9, "gpu_launches": launches * world, "stages": per}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -258,6 +345,16 @@ def run_ours(args):
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def make_train():
+        wl = synth.WORKLOADS[TRAIN_INDEX]
+        t = synth.workload_inputs(TRAIN_INDEX)
+        td = {k: (v.to(dev) if k != "prefix_len" else v) for k, v in t.items()}
+        wts = {k: td[k] for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
+                                  "b_q", "b_k", "b_v", "b_o") if k in td}
+        layer = MotAttnLayer(wts, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_batch=wl.batch,
+                             max_img_tokens=wl.img_tokens, max_prefix=wl.prefix, enable_backward=True)
+        return wl, td, layer
 
     def device_steps(wl, td, layer, steps, warmup, profile):
         x, kc, vc = td["x"], td["k_cache"], td["v_cache"]
@@ -345,6 +442,11 @@ def run_ours(args):
     h2d = (x_h.numel() + kc_h.numel() + vc_h.numel()) * 2
     d2h = y_h.numel() * 2
 
+    # LoRA training step at 2048^2 (forward keeping activations + backward)
+    train = None
+    if not args.skip_train:
+        train = train_steps(make_train(), dev, flush, stream, args, world)
+
     # 1024^2 CFG beside it (same protocol, fewer steps)
     also = None
     if not args.skip_also:
@@ -400,6 +502,7 @@ def run_ours(args):
             "gpu_launches": launches * world,
             "clocks": clk,
             "also": also,
+            "train": train,
         }
         print(json.dumps(line), flush=True)
     layer.close()
@@ -417,6 +520,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-also", action="store_true")
+    ap.add_argument("--skip-train", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--once", action="store_true", help="one warm forward, no timing (ncu target)")

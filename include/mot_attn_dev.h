@@ -32,7 +32,7 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* d, int32_t m, int32
  *   [4] lse     f32 [B, Hq, N]      natural-log softmax normaliser
  *   [5] xhat    [B*N, (Hq+Hkv)*dh]  normalised pre-gain q/k
  *   [6] rstd    f32 [B*N, Hq+Hkv]
- *   [7] u_qkv   bf16 [B*N, 3*RP]    s x A^T per q/k/v (RP = rank rounded up to 64)
+ *   [7] u_qkv   [B*N, 3*RP]         s x A^T per q/k/v (RP = rank rounded up to 64)
  *   [8] u_o     [B*N, RP]           s o A_o^T
  * lcap receives Lcap = round_up(P_max + N, 128). */
 mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32_t img_tokens,

@@ -58,27 +58,6 @@ __global__ void __launch_bounds__(256) build_kv_kernel(const __nv_bfloat16* __re
   if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
 }
 
-// dst[i] = f16(src[i]) for n elements (n % 8 == 0, 16-byte aligned).
-__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src,
-                                                          __half* __restrict__ dst, long long n8, int* status) {
-  bool overflow = false;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 r = reinterpret_cast<const uint4*>(src)[i];
-    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(&r);
-    uint4 o;
-    uint32_t* o32 = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float a = __bfloat162float(bv[2 * k]), b = __bfloat162float(bv[2 * k + 1]);
-      overflow |= fabsf(a) > 65504.f || fabsf(b) > 65504.f;
-      o32[k] = pack_half2(a, b);
-    }
-    reinterpret_cast<uint4*>(dst)[i] = o;
-  }
-  if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
-}
-
 // LoRA bake-in ("SenseNova-U1.5" vLLM-Omni recipe, 8-step distilled LoRA:
 // fused into the gen tower at load):
 //   out[i, j] = RNE_bf16(w[i, j] + s * sum_k b[i, k] a[k, j]),
@@ -107,6 +86,37 @@ __global__ void __launch_bounds__(256) merge_lora_kernel(const __nv_bfloat16* w,
     const long long o = static_cast<long long>(i) * cols + j;
     out[o] = __float2bfloat16_rn(fmaf(s, acc, __bfloat162float(w[o])));
   }
+}
+
+// Several bf16 -> f16 conversions in one launch (LoRA tensors that meet f16
+// activations in an MMA; they may change between calls, so this runs per call).
+struct CvtJobs {
+  const __nv_bfloat16* src[6];
+  __half* dst[6];
+  long long n8[6];  // element count / 8
+  int count;
+};
+
+__global__ void __launch_bounds__(256) cvt_multi_kernel(const CvtJobs jobs, int* status) {
+  bool overflow = false;
+  for (int j = 0; j < jobs.count; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(jobs.src[j]);
+    uint4* dst = reinterpret_cast<uint4*>(jobs.dst[j]);
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < jobs.n8[j];
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+      const uint4 r = src[i];
+      const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&r);
+      float2 f[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[k] = __bfloat1622float2(bv[k]);
+        overflow |= fabsf(f[k].x) > 65504.f || fabsf(f[k].y) > 65504.f;
+      }
+      dst[i] = make_uint4(pack_half2(f[0].x, f[0].y), pack_half2(f[1].x, f[1].y), pack_half2(f[2].x, f[2].y),
+                          pack_half2(f[3].x, f[3].y));
+    }
+  }
+  if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
 }
 
 // f32 copy of a bf16 vector (norm gains)

@@ -28,23 +28,32 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kMaxMaps = 10;
 constexpr int kMaxRegions = 4;
+constexpr int kMaxSegs = 9;
+constexpr uint32_t kMnBoxBytes = 64 * 64 * 2;  // MN-major TMA box: 64 MN x 64 K, 16-bit
 
-struct GemmRegion {
-  int n_begin, n_end;  // D columns [n_begin, n_end); B rows are n - n_begin
-  int b_map;           // maps[] index of the main-segment B tensor
-  int b2_map;          // maps[] index of the extension B tensor (-1: none)
-  int a2_col;          // first A2 column read by this region's extension
+// One K segment: D += A[:, a_k0 + k] B[:, b_k0 + k] over kb 64-wide blocks.
+// A and B may each be K-major (row = M or N index, K contiguous) or MN-major
+// (row = K index, M or N contiguous); MN-major tiles are loaded as 64 x 64
+// TMA boxes and described to the tensor core as transposed operands.
+struct GemmSeg {
+  int a_map;
+  int a_k0[kMaxRegions];   // per N-region (the LoRA extension reads a different u slice per region)
+  int b_map[kMaxRegions];  // per N-region B tensor
+  int b_k0;
+  int kb;
+  uint32_t idesc;
+  int a_mn, b_mn;
 };
 
 struct GemmCore {
-  CUtensorMap maps[kMaxMaps];  // [0] A, [1] A2, [2..] B / B2 tensors
-  GemmRegion regions[kMaxRegions];
+  CUtensorMap maps[kMaxMaps];
+  int region_n0[kMaxRegions + 1];  // region i covers D columns [region_n0[i], region_n0[i+1])
   int num_regions;
+  GemmSeg segs[kMaxSegs];
+  int num_segs;
   int M, N;
-  int kb_main, kb_ext;
   int tiles_m, tiles_n;
-  int b_box_rows;  // rows per B TMA box; BN is a multiple of it
-  uint32_t idesc_main, idesc_ext;
+  int b_box_rows;  // rows per K-major B TMA box; BN is a multiple of it
   int* status;
 };
 
@@ -54,11 +63,11 @@ struct GemmArgs {
   typename Epi::Params epi;
 };
 
-__device__ __forceinline__ const GemmRegion& region_of(const GemmCore& g, int n) {
+__device__ __forceinline__ int region_of(const GemmCore& g, int n) {
   int i = 0;
 #pragma unroll 1
-  while (i + 1 < g.num_regions && n >= g.regions[i].n_end) ++i;
-  return g.regions[i];
+  while (i + 1 < g.num_regions && n >= g.region_n0[i + 1]) ++i;
+  return i;
 }
 
 // grouped tile order: 8 M-tiles share each sweep over N (L2 reuse of A rows)
@@ -87,7 +96,7 @@ struct GemmSmem {
 
 template <int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<Epi> args) {
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128, whole 64-column boxes");
   using L = GemmSmem<BN, STAGES>;
   constexpr uint32_t kTmemCols = tmem_cols_for(2 * BN);
 
@@ -117,10 +126,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    for (int i = 0; i < kMaxMaps; ++i)
-      if (i < 2 + 2 * kMaxRegions) tma_prefetch_desc(&g.maps[i]);
-  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -132,43 +137,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const WaitGuard wg{abort_flag, g.status};
 
   const int num_tiles = g.tiles_m * g.tiles_n;
-  const int kb_total = g.kb_main + g.kb_ext;
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const int boxes = BN / g.b_box_rows;
-      const uint32_t box_bytes = static_cast<uint32_t>(g.b_box_rows) * kBK * 2;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
         const int m0 = tm * kBM, n0 = tn * BN;
-        const GemmRegion& reg0 = region_of(g, n0);
-        for (int kb = 0; kb < kb_total; ++kb) {
-          mbar_wait(&empty[stage], phase ^ 1u, wg);
-          mbar_expect_tx(&full[stage], L::kABytes + L::kBBytes);
-          uint8_t* a_dst = sA + stage * L::kABytes;
-          uint8_t* b_dst = sB + stage * L::kBBytes;
-          if (kb < g.kb_main) {
-            tma_load_2d(a_dst, &g.maps[0], &full[stage], kb * kBK, m0);
-            for (int i = 0; i < boxes; ++i) {
-              const int n = n0 + i * g.b_box_rows;
-              const GemmRegion& r = region_of(g, n);
-              tma_load_2d(b_dst + i * box_bytes, &g.maps[r.b_map], &full[stage], kb * kBK, n - r.n_begin);
+        const int reg0 = region_of(g, n0);
+        for (int si = 0; si < g.num_segs; ++si) {
+          const GemmSeg& sg = g.segs[si];
+          for (int kb = 0; kb < sg.kb; ++kb) {
+            mbar_wait(&empty[stage], phase ^ 1u, wg);
+            mbar_expect_tx(&full[stage], L::kABytes + L::kBBytes);
+            uint8_t* a_dst = sA + stage * L::kABytes;
+            uint8_t* b_dst = sB + stage * L::kBBytes;
+            const int ka = sg.a_k0[reg0] + kb * kBK, kbk = sg.b_k0 + kb * kBK;
+            if (sg.a_mn) {
+              tma_load_2d(a_dst, &g.maps[sg.a_map], &full[stage], m0, ka);
+              tma_load_2d(a_dst + kMnBoxBytes, &g.maps[sg.a_map], &full[stage], m0 + 64, ka);
+            } else {
+              tma_load_2d(a_dst, &g.maps[sg.a_map], &full[stage], ka, m0);
             }
-          } else {
-            const int ke = kb - g.kb_main;
-            tma_load_2d(a_dst, &g.maps[1], &full[stage], reg0.a2_col + ke * kBK, m0);
-            for (int i = 0; i < boxes; ++i) {
-              const int n = n0 + i * g.b_box_rows;
-              const GemmRegion& r = region_of(g, n);
-              tma_load_2d(b_dst + i * box_bytes, &g.maps[r.b2_map], &full[stage], ke * kBK, n - r.n_begin);
+            if (sg.b_mn) {
+              for (int i = 0; i < BN / 64; ++i) {
+                const int n = n0 + i * 64;
+                const int r = region_of(g, n);
+                tma_load_2d(b_dst + i * kMnBoxBytes, &g.maps[sg.b_map[r]], &full[stage], n - g.region_n0[r], kbk);
+              }
+            } else {
+              const uint32_t box_bytes = static_cast<uint32_t>(g.b_box_rows) * kBK * 2;
+              for (int i = 0; i < BN / g.b_box_rows; ++i) {
+                const int n = n0 + i * g.b_box_rows;
+                const int r = region_of(g, n);
+                tma_load_2d(b_dst + i * box_bytes, &g.maps[sg.b_map[r]], &full[stage], kbk, n - g.region_n0[r]);
+              }
             }
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
@@ -183,20 +193,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < kb_total; ++kb) {
-          mbar_wait(&full[stage], phase, wg);
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * L::kBBytes);
-          const uint32_t idesc = kb < g.kb_main ? g.idesc_main : g.idesc_ext;
+        bool first = true;
+        for (int si = 0; si < g.num_segs; ++si) {
+          const GemmSeg& sg = g.segs[si];
+          for (int kb = 0; kb < sg.kb; ++kb) {
+            mbar_wait(&full[stage], phase, wg);
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
+            const uint32_t b_addr = smem_u32(sB + stage * L::kBBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(d_tmem, kmajor_desc(a_addr, kk, L::kABytes), kmajor_desc(b_addr, kk, L::kBBytes), idesc,
-                    (kb | kk) != 0 ? 1u : 0u);
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = sg.a_mn ? mnmajor_desc(a_addr, kk, kMnBoxBytes) : kmajor_desc(a_addr, kk, L::kABytes);
+              const uint64_t bd = sg.b_mn ? mnmajor_desc(b_addr, kk, kMnBoxBytes) : kmajor_desc(b_addr, kk, L::kBBytes);
+              umma_ss(d_tmem, ad, bd, sg.idesc, first ? 0u : 1u);
+              first = false;
+            }
+            umma_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
         umma_commit(&tfull[acc]);
@@ -239,20 +255,76 @@ __device__ __forceinline__ void load_row32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// out = scale * acc, stored as bf16/f16 and/or f32 (f32 optionally added to
-// what is there). Rows >= M and columns >= N are skipped.
+// Up to three 16-bit row-major outputs (each bf16 or f16 with its own scale)
+// and an f32 output (own scale; optionally added to what is there;
+// optionally transposed: element (m, n) at out32[n * ld32 + m]). A 16-bit
+// output may instead hold the rounding residual of another one,
+// bf16(w - float(bf16(w))) with w = acc * that output's scale, so that
+// hi + lo carries about 16 significant bits through two bf16 operands.
+// Rows >= M and columns >= N are skipped.
 struct EpiStore {
+  struct Out16 {
+    void* ptr;
+    long long ld;
+    float scale;
+    int bf16;
+    int residual_of;  // -1, or the index of the output whose residual this is
+  };
   struct Params {
-    void* out16;
-    int out16_bf16;  // 1: bf16, 0: f16
-    long long ld16;
+    Out16 o16[3];
     float* out32;
     long long ld32;
+    float scale32;
     int accumulate32;
-    float scale;
+    int transpose32;
     int M, N;
-    int check_f16;  // flag f16 overflow
+    int check_f16;  // flag f16 overflow of an f16 output
   };
+  __device__ __forceinline__ static uint16_t round16(float w, int is_bf16) {
+    if (is_bf16) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(w);
+      return *reinterpret_cast<const uint16_t*>(&h);
+    }
+    const __half h = __float2half_rn(w);
+    return *reinterpret_cast<const uint16_t*>(&h);
+  }
+  __device__ __forceinline__ static float value16(const Params& p, int i, float acc) {
+    const Out16& o = p.o16[i];
+    if (o.residual_of < 0) return acc * o.scale;
+    const Out16& hi = p.o16[o.residual_of];
+    const float w = acc * hi.scale;
+    const uint16_t r = round16(w, hi.bf16);
+    const float back = hi.bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&r))
+                               : __half2float(*reinterpret_cast<const __half*>(&r));
+    return w - back;
+  }
+  __device__ __forceinline__ static void store16(const Params& p, int i, int m, int n, const float (&v)[32],
+                                                 int ncols, bool& overflow) {
+    const Out16& o = p.o16[i];
+    uint16_t* row = static_cast<uint16_t*>(o.ptr) + m * o.ld + n;
+    if (ncols == 32) {
+      uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a = value16(p, i, v[8 * q + 2 * k]), b = value16(p, i, v[8 * q + 2 * k + 1]);
+          overflow |= p.check_f16 && !o.bf16 && !(fabsf(a) <= 65504.f && fabsf(b) <= 65504.f);
+          w[k] = static_cast<uint32_t>(round16(a, o.bf16)) | (static_cast<uint32_t>(round16(b, o.bf16)) << 16);
+        }
+        dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        if (k >= ncols) continue;
+        const float a = value16(p, i, v[k]);
+        overflow |= p.check_f16 && !o.bf16 && !(fabsf(a) <= 65504.f);
+        row[k] = round16(a, o.bf16);
+      }
+    }
+  }
   template <int BN>
   __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
                                                int* status) {
@@ -262,46 +334,101 @@ struct EpiStore {
     for (int c = 0; c < BN; c += 32) {
       float v[32];
       load_row32(taddr + c, v);
-      if (m >= p.M || n0 + c >= p.N) continue;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= p.scale;
+      const int n = n0 + c;
+      if (m >= p.M || n >= p.N) continue;
+      const int ncols = min(32, p.N - n);
+#pragma unroll 1
+      for (int i = 0; i < 3; ++i)
+        if (p.o16[i].ptr) store16(p, i, m, n, v, ncols, overflow);
       if (p.out32) {
-        float4* dst = reinterpret_cast<float4*>(p.out32 + m * p.ld32 + n0 + c);
+        if (p.transpose32) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float4 w = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          if (p.accumulate32) {
-            const float4 o = dst[i];
-            w.x += o.x;
-            w.y += o.y;
-            w.z += o.z;
-            w.w += o.w;
+          for (int k = 0; k < 32; ++k) {
+            if (k >= ncols) continue;
+            float* o = p.out32 + static_cast<long long>(n + k) * p.ld32 + m;
+            const float w = v[k] * p.scale32;
+            *o = p.accumulate32 ? *o + w : w;
           }
-          dst[i] = w;
+        } else if (ncols == 32) {
+          float4* dst = reinterpret_cast<float4*>(p.out32 + m * p.ld32 + n);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 w = make_float4(v[4 * i] * p.scale32, v[4 * i + 1] * p.scale32, v[4 * i + 2] * p.scale32,
+                                   v[4 * i + 3] * p.scale32);
+            if (p.accumulate32) {
+              const float4 o = dst[i];
+              w.x += o.x;
+              w.y += o.y;
+              w.z += o.z;
+              w.w += o.w;
+            }
+            dst[i] = w;
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            if (k >= ncols) continue;
+            float* o = p.out32 + m * p.ld32 + n + k;
+            const float w = v[k] * p.scale32;
+            *o = p.accumulate32 ? *o + w : w;
+          }
         }
       }
-      if (p.out16) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out16) + m * p.ld16 + n0 + c);
+    }
+    if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
+  }
+};
+
+// Gradient of the attention output: stores dO = acc as f16 [M, Hq*dh] and,
+// per (token, head), D = sum_j dO_j O_j with the forward's attention output O
+// (the rowsum the softmax backward subtracts), taken over the f16-rounded dO
+// the attention backward multiplies. Two heads per 256-column tile.
+struct EpiDattn {
+  struct Params {
+    __half* dout;     // [M, Hq*dh]
+    const __half* o;  // [M, Hq*dh]
+    float* delta;     // [B, Hq, N]
+    int M, N, Hq;
+  };
+  template <int BN>
+  __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
+                                               int* status) {
+    static_assert(BN % 128 == 0, "whole heads per tile");
+    const int m = m0 + row;
+    bool overflow = false;
+#pragma unroll 1
+    for (int hc = 0; hc < BN / 128; ++hc) {
+      float dsum = 0.f;
+      const int head = (n0 >> 7) + hc;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        load_row32(taddr + hc * 128 + c * 32, v);
+        if (m >= p.M) continue;
+        const long long off = static_cast<long long>(m) * p.Hq * 128 + head * 128 + c * 32;
+        const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
+        uint4* d4 = reinterpret_cast<uint4*>(p.dout + off);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          uint4 w;
-          if (p.out16_bf16) {
-            w.x = pack_bf162(v[8 * i + 0], v[8 * i + 1]);
-            w.y = pack_bf162(v[8 * i + 2], v[8 * i + 3]);
-            w.z = pack_bf162(v[8 * i + 4], v[8 * i + 5]);
-            w.w = pack_bf162(v[8 * i + 6], v[8 * i + 7]);
-          } else {
-            w.x = pack_half2(v[8 * i + 0], v[8 * i + 1]);
-            w.y = pack_half2(v[8 * i + 2], v[8 * i + 3]);
-            w.z = pack_half2(v[8 * i + 4], v[8 * i + 5]);
-            w.w = pack_half2(v[8 * i + 6], v[8 * i + 7]);
-          }
-          dst[i] = w;
-        }
-        if (p.check_f16) {
+          const uint4 ow = o4[i];
+          const __half2* oh = reinterpret_cast<const __half2*>(&ow);
+          uint32_t w[4];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) overflow |= fabsf(v[i]) > 65504.f;
+          for (int k = 0; k < 4; ++k) {
+            w[k] = pack_half2(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
+            const float2 df = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+            const float2 of = __half22float2(oh[k]);
+            dsum = fmaf(df.x, of.x, dsum);
+            dsum = fmaf(df.y, of.y, dsum);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) overflow |= !(fabsf(v[8 * i + k]) <= 65504.f);
+          d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
+      }
+      if (m < p.M) {
+        const int b = m / p.N, n = m - b * p.N;
+        p.delta[(static_cast<long long>(b) * p.Hq + head) * p.N + n] = dsum;
       }
     }
     if (overflow) atomicOr(status, DEV_ERR_NUMERIC);

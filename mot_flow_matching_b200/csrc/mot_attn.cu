@@ -1,13 +1,21 @@
 // mot_attn.cu -- C ABI of the gen-tower attention layer (see include/mot_attn.h).
 //
-// Forward launch sequence on the caller's stream (r = LoRA rank):
-//   [r>0] bf16 -> f16 of lora_down/lora_up of o_proj (per call: they may change)
+// Forward launch sequence on the caller's stream (r = LoRA rank, s = alpha/r):
+//   [r>0] A_o -> f16 (it meets the f16 attention output in an MMA)
 //   build_kv      prefix rows of the f16 key/value buffers, zero tail rows
-//   [r>0] lora-down GEMM    u_qkv = s x [A_q; A_k; A_v]^T        (bf16)
+//   [r>0] lora-down GEMM    u_qkv = s x [A_q; A_k; A_v]^T           (bf16)
 //   QKV GEMM + epilogue     x W_qkv^T + u B^T -> RMSNorm -> RoPE -> q^, K, V
-//   attention               o = softmax(q^ K^T / sqrt(dh)) V      (f16)
-//   [r>0] lora-down GEMM    u_o = s o A_o^T                       (f16)
-//   O GEMM                  y = o W_o^T + u_o B_o^T               (bf16 + f32)
+//   attention               o = softmax(q^ K^T / sqrt(dh)) V         (f16)
+//   [r>0] lora-down GEMM    u_o = s o A_o^T                          (bf16)
+//   O GEMM                  y = o W_o^T + u_o B_o^T                  (bf16 + f32)
+// Backward (LoRA training; frozen base, gains and cache):
+//   [r>0] B_q/B_k/B_v -> f16;  g_o = dy B_o
+//   dO GEMM + epilogue      dO = dy W_o + s g_o A_o ; D = rowsum(dO o)
+//   [r>0] dB_o = dy^T u_o ;  dA_o = s g_o^T o
+//   attention backward      dq^ (all keys), dk^, dv (self keys) -> RoPE^-1 ->
+//                           RMSNorm backward -> pre-norm dq, dk, dv (f16)
+//   [r>0] g_j = d{q,k,v} B_j ; dB_j = d{q,k,v}^T u_j ; dA_j = s g_j^T x
+//   dX GEMM                 dx = dq W_q + dk W_k + dv W_v + s sum_j g_j A_j
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -23,6 +31,7 @@
 #include "ptx.cuh"
 #include "gemm.cuh"
 #include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
 #include "aux.cuh"
 
 using namespace mot;
@@ -44,31 +53,40 @@ bool encode_ready() {
   return g_encode != nullptr;
 }
 
-// 2-D map over a row-major [outer, inner] 16-bit tensor with row stride
-// `ld` elements; box = [box_outer rows, 64 columns], 128-byte swizzle.
-bool map2d(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld,
-           uint32_t box_outer) {
-  if (!encode_ready() || inner == 0 || outer == 0) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return g_encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+bool encode(CUtensorMap* m, const void* ptr, bool bf16, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+  if (!encode_ready() || !ptr) return false;
+  for (int i = 0; i < rank; ++i)
+    if (dims[i] == 0) return false;
+  const cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank,
                   const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over a contiguous f16 [outer, mid, 128] tensor, box [1, 128, 64].
-bool map3d_heads(CUtensorMap* m, const void* ptr, uint64_t mid, uint64_t outer) {
-  if (!encode_ready() || mid == 0 || outer == 0) return false;
-  cuuint64_t dims[3] = {128, mid, outer};
-  cuuint64_t strides[2] = {256, mid * 256};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+// K-major operand: row-major [outer, inner] 16-bit tensor (row stride `ld`
+// elements), box = [box_outer rows, 64 columns], 128-byte swizzle.
+bool map2d(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld,
+           uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint32_t box[2] = {64, box_outer};
+  return encode(m, ptr, bf16, 2, dims, strides, box);
+}
+
+// MN-major operand: the same tensor read as 64 x 64 boxes (64 contiguous
+// M/N elements by 64 K rows).
+bool map2d_mn(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld) {
+  return map2d(m, ptr, bf16, inner, outer, ld, 64);
+}
+
+// 3-D map over a contiguous f16 [outer, mid, inner] tensor, box [1, 128, 64].
+bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner * 2, mid * inner * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  return encode(m, ptr, false, 3, dims, strides, box);
 }
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -77,9 +95,15 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // ------------------------------------------------------------------ layouts
 struct Layout {
   int B = 0, N = 0, P = 0, M = 0, Lcap = 0, r = 0, RP = 0;
-  size_t o_q = 0, o_k = 0, o_v = 0, o_attn = 0, o_lse = 0, o_xhat = 0, o_rstd = 0, o_uqkv = 0, o_uo = 0;
-  size_t act_bytes = 0;    // activation region (in `saved`, else in the workspace)
-  size_t w_ao16 = 0, w_bo16 = 0, scratch_bytes = 0;
+  // activations: in `saved` for training, else after the forward scratch
+  size_t o_q = 0, o_k = 0, o_v = 0, o_attn = 0, o_lse = 0, o_xhat = 0, o_rstd = 0, o_uqkv = 0, o_uo = 0,
+         o_uohi = 0, o_uolo = 0, act_bytes = 0;
+  // forward scratch: f16 copies of the LoRA tensors that meet f16 operands
+  size_t w_ao16 = 0, w_bo16 = 0, w_bqkv16 = 0, fwd_scratch = 0;
+  // backward scratch (workspace)
+  size_t b_do = 0, b_delta = 0, b_dqkv = 0, b_gohi = 0, b_golo = 0, b_go16 = 0, b_ghi = 0, b_glo = 0, b_bqkv16 = 0,
+         bwd_scratch = 0;
+  size_t workspace() const { return std::max(fwd_scratch + act_bytes, bwd_scratch); }
 };
 
 Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
@@ -91,7 +115,8 @@ Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
   L.Lcap = static_cast<int>(round_up(static_cast<size_t>(P + N), 128));
   L.r = c.lora_rank;
   L.RP = L.r ? static_cast<int>(round_up(L.r, 64)) : 0;
-  const size_t dh = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M;
+  const size_t dh = c.head_dim, Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M, r = L.r, RP = L.RP;
+  const size_t nqkv = (Hq + 2 * Hkv) * dh;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -105,13 +130,27 @@ Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
   L.o_lse = take(train ? B * Hq * N * 4 : 0);
   L.o_xhat = take(train ? M * (Hq + Hkv) * dh * 2 : 0);
   L.o_rstd = take(train ? M * (Hq + Hkv) * 4 : 0);
-  L.o_uqkv = take(L.r ? M * 3 * L.RP * 2 : 0);
-  L.o_uo = take(L.r ? M * L.RP * 2 : 0);
+  L.o_uqkv = take(r ? M * 3 * RP * 2 : 0);
+  L.o_uo = take(r ? M * RP * 2 : 0);
+  L.o_uohi = take(train && r ? M * RP * 2 : 0);
+  L.o_uolo = take(train && r ? M * RP * 2 : 0);
   L.act_bytes = off;
   off = 0;
-  L.w_ao16 = take(L.r ? L.r * Hq * dh * 2 : 0);
-  L.w_bo16 = take(L.r ? d * L.r * 2 : 0);
-  L.scratch_bytes = off;
+  L.w_ao16 = take(r ? r * Hq * dh * 2 : 0);
+  L.w_bo16 = take(r ? d * r * 2 : 0);
+  L.w_bqkv16 = take(r ? nqkv * r * 2 : 0);
+  L.fwd_scratch = off;
+  off = 0;
+  L.b_do = take(M * Hq * dh * 2);
+  L.b_delta = take(B * Hq * N * 4);
+  L.b_dqkv = take(M * nqkv * 2);
+  L.b_gohi = take(r ? M * RP * 2 : 0);
+  L.b_golo = take(r ? M * RP * 2 : 0);
+  L.b_go16 = take(r ? M * RP * 2 : 0);
+  L.b_ghi = take(r ? M * 3 * RP * 2 : 0);
+  L.b_glo = take(r ? M * 3 * RP * 2 : 0);
+  L.b_bqkv16 = take(r ? nqkv * r * 2 : 0);
+  L.bwd_scratch = c.enable_backward ? off : 0;
   return L;
 }
 
@@ -135,8 +174,6 @@ void set_smem_attr(K kernel, size_t bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
-int g_grid_cap = 0;  // 0 = number of SMs
-
 template <int BN, int STAGES, class Epi>
 cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, int num_sms, cudaStream_t st) {
   static_assert(sizeof(GemmArgs<Epi>) <= 4096, "kernel parameter block");
@@ -149,25 +186,77 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   args.core = core;
   args.epi = ep;
   const int tiles = core.tiles_m * core.tiles_n;
-  const int cap = g_grid_cap > 0 ? g_grid_cap : num_sms;
-  const int grid = std::max(1, std::min(tiles, cap));
+  const int grid = std::max(1, std::min(tiles, num_sms));
   kern<<<grid, kGemmThreads, L::kBytes, st>>>(args);
   return cudaGetLastError();
 }
 
-void core_init(GemmCore& c, int M, int N, int BN, int kb_main, int kb_ext, int b_box_rows, uint32_t idesc_main,
-               uint32_t idesc_ext, int* status) {
+// BN = 64 or 128 instantiation for the narrow (LoRA-rank-wide) GEMMs
+template <class Epi>
+cudaError_t launch_gemm_narrow(int BN, const GemmCore& core, const typename Epi::Params& ep, int num_sms,
+                               cudaStream_t st) {
+  return BN == 64 ? launch_gemm<64, 8, Epi>(core, ep, num_sms, st) : launch_gemm<128, 6, Epi>(core, ep, num_sms, st);
+}
+
+void core_init(GemmCore& c, int M, int N, int BN, int b_box_rows, int* status) {
   std::memset(static_cast<void*>(&c), 0, sizeof(c));
   c.M = M;
   c.N = N;
-  c.kb_main = kb_main;
-  c.kb_ext = kb_ext;
   c.tiles_m = (M + kBM - 1) / kBM;
   c.tiles_n = (N + BN - 1) / BN;
   c.b_box_rows = b_box_rows;
-  c.idesc_main = idesc_main;
-  c.idesc_ext = idesc_ext;
+  c.num_regions = 1;
+  c.region_n0[0] = 0;
+  c.region_n0[1] = N;
   c.status = status;
+}
+
+// one K segment whose A offset and B tensor are the same for every region
+GemmSeg seg1(int a_map, int a_k0, int b_map, int kb, uint32_t idesc, bool a_mn, bool b_mn) {
+  GemmSeg s;
+  std::memset(static_cast<void*>(&s), 0, sizeof(s));
+  s.a_map = a_map;
+  for (int i = 0; i < kMaxRegions; ++i) {
+    s.a_k0[i] = a_k0;
+    s.b_map[i] = b_map;
+  }
+  s.kb = kb;
+  s.idesc = idesc;
+  s.a_mn = a_mn;
+  s.b_mn = b_mn;
+  return s;
+}
+
+EpiStore::Params store_params(int M, int N) {
+  EpiStore::Params p;
+  std::memset(static_cast<void*>(&p), 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.scale32 = 1.0f;
+  for (auto& o : p.o16) {
+    o.scale = 1.0f;
+    o.residual_of = -1;
+  }
+  return p;
+}
+
+void set_out16(EpiStore::Params& p, int i, void* ptr, long long ld, bool bf16, float scale = 1.0f,
+               int residual_of = -1) {
+  p.o16[i].ptr = ptr;
+  p.o16[i].ld = ld;
+  p.o16[i].bf16 = bf16 ? 1 : 0;
+  p.o16[i].scale = scale;
+  p.o16[i].residual_of = residual_of;
+}
+
+// K-major f16 maps over the per-call f16 copies of lora_up (box rows 256)
+bool lora_up16_maps(CUtensorMap* m, const __half* b16, int r, const int (&rows)[3]) {
+  long long off = 0;
+  for (int j = 0; j < 3; ++j) {
+    if (!map2d(&m[j], b16 + off, false, r, rows[j], r, 256)) return false;
+    off += static_cast<long long>(rows[j]) * r;
+  }
+  return true;
 }
 
 }  // namespace
@@ -176,10 +265,14 @@ void core_init(GemmCore& c, int M, int N, int BN, int kb_main, int kb_ext, int b
 constexpr int kMaxStages = 32;
 enum StageId : int {
   ST_CVT_LORA_O = 0, ST_BUILD_KV = 1, ST_LORA_DOWN_QKV = 2, ST_QKV_GEMM = 3, ST_ATTN_FWD = 4,
-  ST_LORA_DOWN_O = 5, ST_O_GEMM = 6,
+  ST_LORA_DOWN_O = 5, ST_O_GEMM = 6, ST_BWD_CVT = 7, ST_BWD_G_O = 8, ST_BWD_DO = 9, ST_BWD_DB_O = 10,
+  ST_BWD_DA_O = 11, ST_BWD_DQ = 12, ST_BWD_DKV = 13, ST_BWD_G_QKV = 14, ST_BWD_DB_QKV = 15, ST_BWD_DA_QKV = 16,
+  ST_BWD_DX = 17,
 };
 const char* const kStageNames[] = {"cvt_lora_o", "build_kv", "lora_down_qkv", "qkv_gemm", "attn_fwd",
-                                   "lora_down_o", "o_gemm"};
+                                   "lora_down_o", "o_gemm", "bwd_cvt_lora", "bwd_g_o", "bwd_do_gemm",
+                                   "bwd_db_o", "bwd_da_o", "attn_bwd_dq", "attn_bwd_dkv", "bwd_g_qkv",
+                                   "bwd_db_qkv", "bwd_da_qkv", "bwd_dx_gemm"};
 
 struct mot_attn {
   mot_attn_config cfg;
@@ -188,7 +281,8 @@ struct mot_attn {
   float scale = 0.f;
   int RP = 0;
   __half* wo16 = nullptr;
-  float* gamma = nullptr;  // [2*dh]: q gain then k gain
+  __half* wqkv16 = nullptr;  // [Hq*dh + 2*Hkv*dh, d] f16 copy of W_q|W_k|W_v (backward)
+  float* gamma = nullptr;    // [2*dh]: q gain then k gain
   float2* rope = nullptr;
   int rope_len = 0;
   int* status = nullptr;
@@ -199,9 +293,11 @@ struct mot_attn {
   cudaEvent_t ev[kMaxStages + 1] = {};
   int stage_ids[kMaxStages] = {};
   int stage_count = 0;
-  CUtensorMap wq, wk, wv, wo;  // base weights, box rows 256
+  // forward weight maps (K-major)
+  CUtensorMap wq, wk, wv, wo;  // box rows 256
   CUtensorMap aq, ak, av;      // lora_down q/k/v, box rows RP
-  CUtensorMap bq, bk, bv;      // lora_up q/k/v, box rows 256
+  // backward weight maps (MN-major, 64 x 64 boxes)
+  CUtensorMap wo_mn, ao_mn, bo_mn, wq16_mn, wk16_mn, wv16_mn, aq_mn, ak_mn, av_mn;
 };
 
 namespace {
@@ -215,10 +311,45 @@ mot_status build_weight_maps(mot_attn* h) {
     const uint64_t r = h->rank;
     const uint32_t box_a = static_cast<uint32_t>(h->RP);
     ok = map2d(&h->aq, h->w.a_q, true, d, r, d, box_a) && map2d(&h->ak, h->w.a_k, true, d, r, d, box_a) &&
-         map2d(&h->av, h->w.a_v, true, d, r, d, box_a) && map2d(&h->bq, h->w.b_q, true, r, qd, r, 256) &&
-         map2d(&h->bk, h->w.b_k, true, r, kvd, r, 256) && map2d(&h->bv, h->w.b_v, true, r, kvd, r, 256);
+         map2d(&h->av, h->w.a_v, true, d, r, d, box_a);
+  }
+  if (ok && c.enable_backward) {
+    ok = map2d_mn(&h->wo_mn, h->w.w_o, true, qd, d, qd) && map2d_mn(&h->wq16_mn, h->wqkv16, false, d, qd, d) &&
+         map2d_mn(&h->wk16_mn, h->wqkv16 + qd * d, false, d, kvd, d) &&
+         map2d_mn(&h->wv16_mn, h->wqkv16 + (qd + kvd) * d, false, d, kvd, d);
+    if (ok && h->rank > 0) {
+      const uint64_t r = h->rank;
+      ok = map2d_mn(&h->ao_mn, h->w.a_o, true, qd, r, qd) && map2d_mn(&h->bo_mn, h->w.b_o, true, r, d, r) &&
+           map2d_mn(&h->aq_mn, h->w.a_q, true, d, r, d) && map2d_mn(&h->ak_mn, h->w.a_k, true, d, r, d) &&
+           map2d_mn(&h->av_mn, h->w.a_v, true, d, r, d);
+    }
   }
   return ok ? MOT_OK : MOT_ERR_CUDA;
+}
+
+// f16 copies the handle keeps of frozen weights (W_o always; W_q|W_k|W_v for backward)
+cudaError_t refresh_f16_copies(mot_attn* h, cudaStream_t s) {
+  const mot_attn_config& c = h->cfg;
+  const long long d = c.hidden, qd = c.n_q_heads * 128, kvd = c.n_kv_heads * 128;
+  CvtJobs jobs{};
+  jobs.src[0] = static_cast<const __nv_bfloat16*>(h->w.w_o);
+  jobs.dst[0] = h->wo16;
+  jobs.n8[0] = d * qd / 8;
+  jobs.count = 1;
+  if (c.enable_backward) {
+    const void* src[3] = {h->w.w_q, h->w.w_k, h->w.w_v};
+    const long long rows[3] = {qd, kvd, kvd};
+    long long off = 0;
+    for (int i = 0; i < 3; ++i) {
+      jobs.src[1 + i] = static_cast<const __nv_bfloat16*>(src[i]);
+      jobs.dst[1 + i] = h->wqkv16 + off;
+      jobs.n8[1 + i] = rows[i] * d / 8;
+      off += rows[i] * d;
+    }
+    jobs.count = 4;
+  }
+  cvt_multi_kernel<<<4 * h->num_sms, 256, 0, s>>>(jobs, h->status);
+  return cudaGetLastError();
 }
 
 void release(mot_attn* h) {
@@ -226,11 +357,38 @@ void release(mot_attn* h) {
   for (cudaEvent_t e : h->ev)
     if (e) cudaEventDestroy(e);
   cudaFree(h->wo16);
+  cudaFree(h->wqkv16);
   cudaFree(h->gamma);
   cudaFree(h->rope);
   cudaFree(h->status);
   delete h;
 }
+
+// launch bookkeeping shared by forward and backward: error capture, launch
+// count and the optional per-launch events
+struct Launches {
+  mot_attn* h;
+  cudaStream_t st;
+  int count = 0;
+  int stage = 0;
+  cudaError_t err = cudaSuccess;
+  Launches(mot_attn* handle, cudaStream_t s) : h(handle), st(s) {
+    if (h->profile) cudaEventRecord(h->ev[0], st);
+  }
+  void done(cudaError_t e) {
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    if (h->profile && count < kMaxStages) {
+      h->stage_ids[count] = stage;
+      cudaEventRecord(h->ev[count + 1], st);
+    }
+    ++count;
+  }
+  mot_status finish() {
+    h->last_launches = count;
+    h->stage_count = std::min(count, kMaxStages);
+    return err == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+  }
+};
 
 }  // namespace
 
@@ -260,7 +418,7 @@ mot_status mot_attn_query_sizes(const mot_attn_config* cfg, int32_t batch, int32
     return MOT_ERR_UNSUPPORTED_SHAPE;
   const Layout inf = make_layout(*cfg, batch, img_tokens, prefix_max, false);
   const Layout trn = make_layout(*cfg, batch, img_tokens, prefix_max, true);
-  if (workspace_bytes) *workspace_bytes = inf.scratch_bytes + inf.act_bytes;
+  if (workspace_bytes) *workspace_bytes = std::max({inf.fwd_scratch + inf.act_bytes, trn.fwd_scratch, trn.bwd_scratch});
   if (saved_bytes) *saved_bytes = trn.act_bytes;
   return MOT_OK;
 }
@@ -293,11 +451,12 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  const size_t dh = cfg->head_dim, d = cfg->hidden, qd = cfg->n_q_heads * dh;
+  const size_t dh = cfg->head_dim, d = cfg->hidden, qd = cfg->n_q_heads * dh, kvd = cfg->n_kv_heads * dh;
   h->rope_len = cfg->max_prefix + cfg->max_img_tokens;
   bool ok = cudaMalloc(&h->wo16, d * qd * 2) == cudaSuccess && cudaMalloc(&h->gamma, 2 * dh * 4) == cudaSuccess &&
             cudaMalloc(&h->rope, static_cast<size_t>(h->rope_len) * 64 * sizeof(float2)) == cudaSuccess &&
             cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
+  if (ok && cfg->enable_backward) ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess;
   if (!ok) {
     release(h);
     return MOT_ERR_CUDA;
@@ -313,9 +472,8 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
        cudaMemsetAsync(h->status, 0, sizeof(int), s) == cudaSuccess;
   bf16_to_f32_kernel<<<1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(wts->q_norm), h->gamma, 128);
   bf16_to_f32_kernel<<<1, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(wts->k_norm), h->gamma + 128, 128);
-  bf16_to_f16_kernel<<<2 * h->num_sms, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(wts->w_o), h->wo16,
-                                                     static_cast<long long>(d * qd / 8), h->status);
-  ok = ok && cudaGetLastError() == cudaSuccess && cudaStreamSynchronize(s) == cudaSuccess;
+  ok = ok && cudaGetLastError() == cudaSuccess && refresh_f16_copies(h, s) == cudaSuccess &&
+       cudaStreamSynchronize(s) == cudaSuccess;
   if (ok) ok = build_weight_maps(h) == MOT_OK;
   if (!ok) {
     release(h);
@@ -358,11 +516,11 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   const bool train = saved != nullptr;
   const Layout L = make_layout(c, B, N, P, train);
   if (train && saved_bytes < L.act_bytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
-  if (workspace_bytes < L.scratch_bytes + (train ? 0 : L.act_bytes)) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < L.fwd_scratch + (train ? 0 : L.act_bytes)) return MOT_ERR_WORKSPACE_TOO_SMALL;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* act = train ? static_cast<uint8_t*>(saved) : ws + L.scratch_bytes;
+  uint8_t* act = train ? static_cast<uint8_t*>(saved) : ws + L.fwd_scratch;
   __half* q_hat = reinterpret_cast<__half*>(act + L.o_q);
   __half* k_all = reinterpret_cast<__half*>(act + L.o_k);
   __half* v_all = reinterpret_cast<__half*>(act + L.o_v);
@@ -370,38 +528,41 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   float* lse = train ? reinterpret_cast<float*>(act + L.o_lse) : nullptr;
   __half* xhat = train ? reinterpret_cast<__half*>(act + L.o_xhat) : nullptr;
   float* rstd = train ? reinterpret_cast<float*>(act + L.o_rstd) : nullptr;
-  __nv_bfloat16* u_qkv = reinterpret_cast<__nv_bfloat16*>(act + L.o_uqkv);
+  __half* u_qkv = reinterpret_cast<__half*>(act + L.o_uqkv);
   __half* u_o = reinterpret_cast<__half*>(act + L.o_uo);
+  __nv_bfloat16* u_ohi = train ? reinterpret_cast<__nv_bfloat16*>(act + L.o_uohi) : nullptr;
+  __nv_bfloat16* u_olo = train ? reinterpret_cast<__nv_bfloat16*>(act + L.o_uolo) : nullptr;
   __half* ao16 = reinterpret_cast<__half*>(ws + L.w_ao16);
   __half* bo16 = reinterpret_cast<__half*>(ws + L.w_bo16);
+  __half* bqkv16 = reinterpret_cast<__half*>(ws + L.w_bqkv16);
 
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M, r = h->rank, RP = h->RP;
   const int qd = Hq * 128, kvd = Hkv * 128, nqkv = qd + 2 * kvd;
-  int launches = 0;
-  cudaError_t e = cudaSuccess;
-  int stage = 0;
-  if (h->profile) cudaEventRecord(h->ev[0], st);
-  auto chk = [&](cudaError_t err) {
-    if (err != cudaSuccess && e == cudaSuccess) e = err;
-    if (h->profile && launches < kMaxStages) {
-      h->stage_ids[launches] = stage;
-      cudaEventRecord(h->ev[launches + 1], st);
-    }
-    ++launches;
-  };
+  Launches lz(h, st);
 
-  // 1. o-side LoRA tensors to f16 (they share the MMA with f16 activations)
-  stage = ST_CVT_LORA_O;
+  // 1. f16 copies of A_o and of every lora_up (they meet f16 operands); per
+  //    call, since a trainer updates them in place between calls
+  const int outj[3] = {qd, kvd, kvd};
+  lz.stage = ST_CVT_LORA_O;
   if (r > 0) {
-    bf16_to_f16_kernel<<<64, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h->w.a_o), ao16,
-                                           static_cast<long long>(r) * qd / 8, h->status);
-    chk(cudaGetLastError());
-    bf16_to_f16_kernel<<<64, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h->w.b_o), bo16,
-                                           static_cast<long long>(d) * r / 8, h->status);
-    chk(cudaGetLastError());
+    CvtJobs jobs{};
+    const void* src[5] = {h->w.a_o, h->w.b_o, h->w.b_q, h->w.b_k, h->w.b_v};
+    __half* dst[5] = {ao16, bo16, bqkv16, bqkv16 + static_cast<long long>(qd) * r,
+                      bqkv16 + static_cast<long long>(qd + kvd) * r};
+    const long long n[5] = {static_cast<long long>(r) * qd, static_cast<long long>(d) * r,
+                            static_cast<long long>(qd) * r, static_cast<long long>(kvd) * r,
+                            static_cast<long long>(kvd) * r};
+    for (int i = 0; i < 5; ++i) {
+      jobs.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
+      jobs.dst[i] = dst[i];
+      jobs.n8[i] = n[i] / 8;
+    }
+    jobs.count = 5;
+    cvt_multi_kernel<<<2 * h->num_sms, 256, 0, st>>>(jobs, h->status);
+    lz.done(cudaGetLastError());
   }
   // 2. key/value buffers: prefix rows + zero tail
-  stage = ST_BUILD_KV;
+  lz.stage = ST_BUILD_KV;
   {
     PlenArray pl{};
     for (int b = 0; b < B; ++b) pl.v[b] = prefix_len[b];
@@ -410,47 +571,60 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     build_kv_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_cache),
                                           static_cast<const __nv_bfloat16*>(v_cache), k_all, v_all, Hkv,
                                           std::max(P, 1), N, L.Lcap, chunks, pl, h->status);
-    chk(cudaGetLastError());
+    lz.done(cudaGetLastError());
   }
-  // 3. LoRA down for q/k/v: u_qkv[:, j*RP:(j+1)*RP] = s x A_j^T
-  stage = ST_LORA_DOWN_QKV;
+  // 3. LoRA down for q/k/v: u_qkv[:, j*RP:(j+1)*RP] = s x A_j^T (f16)
+  lz.stage = ST_LORA_DOWN_QKV;
   if (r > 0) {
     GemmCore core;
     const int BN = RP == 64 ? 192 : 128;
-    core_init(core, M, 3 * RP, BN, d / 64, 0, RP, idesc_f16(128, BN, true, true), 0, h->status);
-    bool ok = map2d(&core.maps[0], x, true, d, M, d, 128);
+    core_init(core, M, 3 * RP, BN, RP, h->status);
+    if (!map2d(&core.maps[0], x, true, d, M, d, 128)) return MOT_ERR_CUDA;
     core.maps[2] = h->aq;
     core.maps[3] = h->ak;
     core.maps[4] = h->av;
     core.num_regions = 3;
-    for (int j = 0; j < 3; ++j) core.regions[j] = GemmRegion{j * RP, (j + 1) * RP, 2 + j, -1, 0};
-    EpiStore::Params ep{u_qkv, 1, 3 * RP, nullptr, 0, 0, h->scale, M, 3 * RP, 0};
-    if (!ok) return MOT_ERR_CUDA;
+    for (int j = 0; j <= 3; ++j) core.region_n0[j] = j * RP;
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, BN, true, true), false, false);
+    for (int j = 0; j < 3; ++j) core.segs[0].b_map[j] = 2 + j;
+    core.num_segs = 1;
+    EpiStore::Params ep = store_params(M, 3 * RP);
+    set_out16(ep, 0, u_qkv, 3 * RP, false, h->scale);
+    ep.check_f16 = 1;
     if (BN == 192)
-      chk(launch_gemm<192, 5, EpiStore>(core, ep, h->num_sms, st));
+      lz.done(launch_gemm<192, 5, EpiStore>(core, ep, h->num_sms, st));
     else
-      chk(launch_gemm<128, 6, EpiStore>(core, ep, h->num_sms, st));
+      lz.done(launch_gemm<128, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   // 4. QKV projection (+ LoRA up) with RMSNorm + RoPE epilogue
-  stage = ST_QKV_GEMM;
+  lz.stage = ST_QKV_GEMM;
   {
     GemmCore core;
-    core_init(core, M, nqkv, 256, d / 64, r > 0 ? RP / 64 : 0, 256, idesc_f16(128, 256, true, true),
-              idesc_f16(128, 256, true, true), h->status);
+    core_init(core, M, nqkv, 256, 256, h->status);
     bool ok = map2d(&core.maps[0], x, true, d, M, d, 128);
-    if (r > 0) ok = ok && map2d(&core.maps[1], u_qkv, true, 3 * RP, M, 3 * RP, 128);
+    if (r > 0)
+      ok = ok && map2d(&core.maps[1], u_qkv, false, 3 * RP, M, 3 * RP, 128) &&
+           lora_up16_maps(&core.maps[5], bqkv16, r, outj);
+    if (!ok) return MOT_ERR_CUDA;
     core.maps[2] = h->wq;
     core.maps[3] = h->wk;
     core.maps[4] = h->wv;
-    if (r > 0) {
-      core.maps[5] = h->bq;
-      core.maps[6] = h->bk;
-      core.maps[7] = h->bv;
-    }
     core.num_regions = 3;
-    core.regions[0] = GemmRegion{0, qd, 2, r > 0 ? 5 : -1, 0};
-    core.regions[1] = GemmRegion{qd, qd + kvd, 3, r > 0 ? 6 : -1, RP};
-    core.regions[2] = GemmRegion{qd + kvd, nqkv, 4, r > 0 ? 7 : -1, 2 * RP};
+    core.region_n0[0] = 0;
+    core.region_n0[1] = qd;
+    core.region_n0[2] = qd + kvd;
+    core.region_n0[3] = nqkv;
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, 256, true, true), false, false);
+    for (int j = 0; j < 3; ++j) core.segs[0].b_map[j] = 2 + j;
+    core.num_segs = 1;
+    if (r > 0) {
+      core.segs[1] = seg1(1, 0, 5, RP / 64, idesc_f16(128, 256, false, false), false, false);
+      for (int j = 0; j < 3; ++j) {
+        core.segs[1].a_k0[j] = j * RP;
+        core.segs[1].b_map[j] = 5 + j;
+      }
+      core.num_segs = 2;
+    }
     EpiQkv::Params ep{};
     ep.q_out = q_hat;
     ep.k_out = k_all;
@@ -467,17 +641,16 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ep.Lcap = L.Lcap;
     ep.M = M;
     ep.eps = c.rms_eps;
-    if (!ok) return MOT_ERR_CUDA;
-    chk(launch_gemm<256, 4, EpiQkv>(core, ep, h->num_sms, st));
+    lz.done(launch_gemm<256, 4, EpiQkv>(core, ep, h->num_sms, st));
   }
   // 5. attention
-  stage = ST_ATTN_FWD;
+  lz.stage = ST_ATTN_FWD;
   {
     AttnFwdParams ap{};
-    bool ok = map3d_heads(&ap.q_map, q_hat, N, static_cast<uint64_t>(B) * Hq) &&
-              map3d_heads(&ap.k_map, k_all, L.Lcap, static_cast<uint64_t>(B) * Hkv) &&
-              map3d_heads(&ap.v_map, v_all, L.Lcap, static_cast<uint64_t>(B) * Hkv);
-    if (!ok) return MOT_ERR_CUDA;
+    if (!map3d(&ap.q_map, q_hat, 128, N, static_cast<uint64_t>(B) * Hq) ||
+        !map3d(&ap.k_map, k_all, 128, L.Lcap, static_cast<uint64_t>(B) * Hkv) ||
+        !map3d(&ap.v_map, v_all, 128, L.Lcap, static_cast<uint64_t>(B) * Hkv))
+      return MOT_ERR_CUDA;
     ap.B = B;
     ap.N = N;
     ap.Hq = Hq;
@@ -492,54 +665,315 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(attn_fwd_kernel, AttnSmem::kBytes); });
     attn_fwd_kernel<<<B * Hq * ap.q_tiles, kAttnThreads, AttnSmem::kBytes, st>>>(ap);
-    chk(cudaGetLastError());
+    lz.done(cudaGetLastError());
   }
-  // 6. LoRA down for o: u_o = s o A_o^T (f16)
-  stage = ST_LORA_DOWN_O;
+  // 6. LoRA down for o: u_o = s o A_o^T (f16; training also keeps it as a bf16 hi + lo pair)
+  lz.stage = ST_LORA_DOWN_O;
   if (r > 0) {
     GemmCore core;
-    core_init(core, M, RP, RP, qd / 64, 0, RP, idesc_f16(128, RP, false, false), 0, h->status);
-    bool ok = map2d(&core.maps[0], attn, false, qd, M, qd, 128) &&
-              map2d(&core.maps[2], ao16, false, qd, r, qd, RP);
-    core.num_regions = 1;
-    core.regions[0] = GemmRegion{0, RP, 2, -1, 0};
-    EpiStore::Params ep{u_o, 0, RP, nullptr, 0, 0, h->scale, M, RP, 1};
-    if (!ok) return MOT_ERR_CUDA;
-    if (RP == 64)
-      chk(launch_gemm<64, 8, EpiStore>(core, ep, h->num_sms, st));
-    else
-      chk(launch_gemm<128, 6, EpiStore>(core, ep, h->num_sms, st));
+    core_init(core, M, RP, RP, RP, h->status);
+    if (!map2d(&core.maps[0], attn, false, qd, M, qd, 128) || !map2d(&core.maps[2], ao16, false, qd, r, qd, RP))
+      return MOT_ERR_CUDA;
+    core.segs[0] = seg1(0, 0, 2, qd / 64, idesc_f16(128, RP, false, false), false, false);
+    core.num_segs = 1;
+    EpiStore::Params ep = store_params(M, RP);
+    set_out16(ep, 0, u_o, RP, false, h->scale);
+    if (train) {
+      set_out16(ep, 1, u_ohi, RP, true, h->scale);
+      set_out16(ep, 2, u_olo, RP, true, 1.0f, 1);
+    }
+    ep.check_f16 = 1;
+    lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
   }
   // 7. O projection (+ LoRA up): y bf16 and optional f32
-  stage = ST_O_GEMM;
+  lz.stage = ST_O_GEMM;
   {
     GemmCore core;
-    core_init(core, M, d, 256, qd / 64, r > 0 ? RP / 64 : 0, 256, idesc_f16(128, 256, false, false),
-              idesc_f16(128, 256, false, false), h->status);
+    core_init(core, M, d, 256, 256, h->status);
     bool ok = map2d(&core.maps[0], attn, false, qd, M, qd, 128);
-    if (r > 0) ok = ok && map2d(&core.maps[1], u_o, false, RP, M, RP, 128) && map2d(&core.maps[3], bo16, false, r, d, r, 256);
-    core.maps[2] = h->wo;
-    core.num_regions = 1;
-    core.regions[0] = GemmRegion{0, d, 2, r > 0 ? 3 : -1, 0};
-    EpiStore::Params ep{y, 1, d, y_f32, d, 0, 1.0f, M, d, 0};
+    if (r > 0)
+      ok = ok && map2d(&core.maps[1], u_o, false, RP, M, RP, 128) && map2d(&core.maps[3], bo16, false, r, d, r, 256);
     if (!ok) return MOT_ERR_CUDA;
-    chk(launch_gemm<256, 4, EpiStore>(core, ep, h->num_sms, st));
+    core.maps[2] = h->wo;
+    core.segs[0] = seg1(0, 0, 2, qd / 64, idesc_f16(128, 256, false, false), false, false);
+    core.num_segs = 1;
+    if (r > 0) {
+      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(128, 256, false, false), false, false);
+      core.num_segs = 2;
+    }
+    EpiStore::Params ep = store_params(M, d);
+    set_out16(ep, 0, y, d, true);
+    ep.out32 = y_f32;
+    ep.ld32 = d;
+    lz.done(launch_gemm<256, 4, EpiStore>(core, ep, h->num_sms, st));
   }
-  h->last_launches = launches;
-  h->stage_count = std::min(launches, kMaxStages);
-  return e == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+  return lz.finish();
 }
 
 mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_t B, int32_t N, const void* k_cache,
                              const void* v_cache, const int32_t* prefix_len, int32_t P, const void* saved,
                              size_t saved_bytes, void* dx, float* dx_f32, float* const d_a[4], float* const d_b[4],
                              int32_t accumulate, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)dy; (void)x; (void)B; (void)N; (void)k_cache; (void)v_cache; (void)prefix_len; (void)P; (void)saved_bytes;
-  (void)dx; (void)dx_f32; (void)d_a; (void)d_b; (void)accumulate; (void)workspace; (void)workspace_bytes;
-  (void)stream;
-  if (!h) return MOT_ERR_INVALID_ARGUMENT;
+  (void)k_cache;
+  (void)v_cache;  // the forward left the f16 key/value buffers in `saved`
+  if (!h || !dy || !x || !dx || !prefix_len || !workspace) return MOT_ERR_INVALID_ARGUMENT;
   if (!saved) return MOT_ERR_NO_SAVED_STATE;
-  return MOT_ERR_UNSUPPORTED_SHAPE;
+  const mot_attn_config& c = h->cfg;
+  if (!c.enable_backward) return MOT_ERR_INVALID_ARGUMENT;
+  if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
+  if (B > c.max_batch || N > c.max_img_tokens || P > c.max_prefix) return MOT_ERR_UNSUPPORTED_SHAPE;
+  for (int b = 0; b < B; ++b)
+    if (prefix_len[b] < 0 || prefix_len[b] > P) return MOT_ERR_INVALID_ARGUMENT;
+  const int r = h->rank;
+  if (r > 0) {
+    if (!d_a || !d_b) return MOT_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < 4; ++i)
+      if (!d_a[i] || !d_b[i] || !aligned16(d_a[i]) || !aligned16(d_b[i])) return d_a[i] && d_b[i] ? MOT_ERR_ALIGNMENT : MOT_ERR_INVALID_ARGUMENT;
+  }
+  const void* ptrs[] = {dy, x, dx, dx_f32, saved, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOT_ERR_ALIGNMENT;
+  const Layout L = make_layout(c, B, N, P, true);
+  if (saved_bytes < L.act_bytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < L.bwd_scratch) return MOT_ERR_WORKSPACE_TOO_SMALL;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* act = static_cast<const uint8_t*>(saved);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const __half* q_hat = reinterpret_cast<const __half*>(act + L.o_q);
+  const __half* k_all = reinterpret_cast<const __half*>(act + L.o_k);
+  const __half* v_all = reinterpret_cast<const __half*>(act + L.o_v);
+  const __half* attn = reinterpret_cast<const __half*>(act + L.o_attn);
+  const float* lse = reinterpret_cast<const float*>(act + L.o_lse);
+  const __half* xhat = reinterpret_cast<const __half*>(act + L.o_xhat);
+  const float* rstd = reinterpret_cast<const float*>(act + L.o_rstd);
+  const __half* u_qkv = reinterpret_cast<const __half*>(act + L.o_uqkv);          // s x A_j^T
+  const __nv_bfloat16* u_ohi = reinterpret_cast<const __nv_bfloat16*>(act + L.o_uohi);  // s o A_o^T, hi + lo
+  const __nv_bfloat16* u_olo = reinterpret_cast<const __nv_bfloat16*>(act + L.o_uolo);
+  __half* dO = reinterpret_cast<__half*>(ws + L.b_do);
+  float* delta = reinterpret_cast<float*>(ws + L.b_delta);
+  __half* dqkv = reinterpret_cast<__half*>(ws + L.b_dqkv);
+  // s g as bf16 hi + lo pairs (they meet bf16 x and lora_down), s g_o also in f16
+  __nv_bfloat16* g_ohi = reinterpret_cast<__nv_bfloat16*>(ws + L.b_gohi);
+  __nv_bfloat16* g_olo = reinterpret_cast<__nv_bfloat16*>(ws + L.b_golo);
+  __half* g_o16 = reinterpret_cast<__half*>(ws + L.b_go16);
+  __nv_bfloat16* g_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.b_ghi);
+  __nv_bfloat16* g_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.b_glo);
+  __half* b16 = reinterpret_cast<__half*>(ws + L.b_bqkv16);  // B_q|B_k|B_v in f16
+
+  const int Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M, RP = h->RP;
+  const int qd = Hq * 128, kvd = Hkv * 128, nqkv = qd + 2 * kvd;
+  const int kb_tok = (M + 63) / 64;  // K blocks over tokens (zero-filled tail)
+  const int col0[3] = {0, qd, qd + kvd}, outj[3] = {qd, kvd, kvd};
+  Launches lz(h, st);
+
+  if (r > 0) {
+    // B_q, B_k, B_v to f16 (they meet the f16 pre-norm gradients)
+    lz.stage = ST_BWD_CVT;
+    CvtJobs jobs{};
+    const void* src[3] = {h->w.b_q, h->w.b_k, h->w.b_v};
+    for (int j = 0; j < 3; ++j) {
+      jobs.src[j] = static_cast<const __nv_bfloat16*>(src[j]);
+      jobs.dst[j] = b16 + static_cast<long long>(col0[j]) * r;
+      jobs.n8[j] = static_cast<long long>(outj[j]) * r / 8;
+    }
+    jobs.count = 3;
+    cvt_multi_kernel<<<64, 256, 0, st>>>(jobs, h->status);
+    lz.done(cudaGetLastError());
+    // g_o = dy B_o  -> s g_o as bf16 hi + lo, and as f16
+    lz.stage = ST_BWD_G_O;
+    GemmCore core;
+    core_init(core, M, RP, RP, RP, h->status);
+    if (!map2d(&core.maps[0], dy, true, d, M, d, 128)) return MOT_ERR_CUDA;
+    core.maps[2] = h->bo_mn;
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, RP, true, true, false, true), false, true);
+    core.num_segs = 1;
+    EpiStore::Params ep = store_params(M, RP);
+    set_out16(ep, 0, g_ohi, RP, true, h->scale);
+    set_out16(ep, 1, g_olo, RP, true, 1.0f, 0);
+    set_out16(ep, 2, g_o16, RP, false, h->scale);
+    ep.check_f16 = 1;
+    lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+  }
+  // dO = dy W_o + s g_o A_o (f16) and D = rowsum(dO o)
+  lz.stage = ST_BWD_DO;
+  {
+    GemmCore core;
+    core_init(core, M, qd, 256, 256, h->status);
+    bool ok = map2d(&core.maps[0], dy, true, d, M, d, 128);
+    if (r > 0)
+      ok = ok && map2d(&core.maps[1], g_ohi, true, RP, M, RP, 128) && map2d(&core.maps[4], g_olo, true, RP, M, RP, 128);
+    if (!ok) return MOT_ERR_CUDA;
+    core.maps[2] = h->wo_mn;
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+    core.num_segs = 1;
+    if (r > 0) {
+      core.maps[3] = h->ao_mn;
+      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+      core.segs[2] = seg1(4, 0, 3, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+      core.num_segs = 3;
+    }
+    EpiDattn::Params ep{dO, attn, delta, M, N, Hq};
+    lz.done(launch_gemm<256, 4, EpiDattn>(core, ep, h->num_sms, st));
+  }
+  if (r > 0) {
+    // dB_o = dy^T u_o   [d, r], with u_o as its bf16 hi + lo pair
+    lz.stage = ST_BWD_DB_O;
+    {
+      GemmCore core;
+      core_init(core, d, RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], dy, true, d, M, d) || !map2d_mn(&core.maps[2], u_ohi, true, RP, M, RP) ||
+          !map2d_mn(&core.maps[3], u_olo, true, RP, M, RP))
+        return MOT_ERR_CUDA;
+      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
+      core.segs[1] = seg1(0, 0, 3, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
+      core.num_segs = 2;
+      EpiStore::Params ep = store_params(d, r);
+      ep.out32 = d_b[3];
+      ep.ld32 = r;
+      ep.accumulate32 = accumulate;
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+    }
+    // dA_o = (s g_o)^T o   [r, qd], computed as its transpose o^T (s g_o)
+    lz.stage = ST_BWD_DA_O;
+    {
+      GemmCore core;
+      core_init(core, qd, RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], attn, false, qd, M, qd) || !map2d_mn(&core.maps[2], g_o16, false, RP, M, RP))
+        return MOT_ERR_CUDA;
+      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, false, false, true, true), true, true);
+      core.num_segs = 1;
+      EpiStore::Params ep = store_params(qd, r);
+      ep.out32 = d_a[3];
+      ep.ld32 = qd;
+      ep.accumulate32 = accumulate;
+      ep.transpose32 = 1;
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+    }
+  }
+  // attention backward: dq^ over all keys, dk^, dv over the self keys
+  {
+    AttnBwdParams ap{};
+    if (!map3d(&ap.q_map, q_hat, 128, N, static_cast<uint64_t>(B) * Hq) ||
+        !map3d(&ap.k_map, k_all, 128, L.Lcap, static_cast<uint64_t>(B) * Hkv) ||
+        !map3d(&ap.v_map, v_all, 128, L.Lcap, static_cast<uint64_t>(B) * Hkv) ||
+        !map3d(&ap.do_map, dO, qd, N, B))
+      return MOT_ERR_CUDA;
+    ap.B = B;
+    ap.N = N;
+    ap.Hq = Hq;
+    ap.Hkv = Hkv;
+    ap.Lcap = L.Lcap;
+    ap.q_tiles = (N + 127) / 128;
+    ap.kv_tiles = (N + 127) / 128;
+    for (int b = 0; b < B; ++b) ap.plen[b] = prefix_len[b];
+    ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+    ap.inv_sqrt_dh = static_cast<float>(1.0 / std::sqrt(128.0));
+    ap.lse = lse;
+    ap.delta = delta;
+    ap.xhat = xhat;
+    ap.rstd = rstd;
+    ap.gamma_q = h->gamma;
+    ap.gamma_k = h->gamma + 128;
+    ap.rope = h->rope;
+    ap.dqkv = dqkv;
+    ap.status = h->status;
+    static std::once_flag once;
+    std::call_once(once, [] {
+      set_smem_attr(attn_bwd_dq_kernel, AttnBwdSmem::kBytes);
+      set_smem_attr(attn_bwd_dkv_kernel, AttnBwdSmem::kBytes);
+    });
+    lz.stage = ST_BWD_DQ;
+    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, 192, AttnBwdSmem::kBytes, st>>>(ap);
+    lz.done(cudaGetLastError());
+    lz.stage = ST_BWD_DKV;
+    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, 192, AttnBwdSmem::kBytes, st>>>(ap);
+    lz.done(cudaGetLastError());
+  }
+  if (r > 0) {
+    for (int j = 0; j < 3; ++j) {
+      // g_j = d{q,k,v}_pre B_j  -> s g_j as bf16 hi + lo in columns [j*RP, (j+1)*RP)
+      lz.stage = ST_BWD_G_QKV;
+      GemmCore core;
+      core_init(core, M, RP, RP, RP, h->status);
+      if (!map2d(&core.maps[0], dqkv, false, nqkv, M, nqkv, 128) ||
+          !map2d_mn(&core.maps[2], b16 + static_cast<long long>(col0[j]) * r, false, r, outj[j], r))
+        return MOT_ERR_CUDA;
+      core.segs[0] = seg1(0, col0[j], 2, outj[j] / 64, idesc_f16(128, RP, false, false, false, true), false, true);
+      core.num_segs = 1;
+      EpiStore::Params ep = store_params(M, RP);
+      set_out16(ep, 0, g_hi + j * RP, 3 * RP, true, h->scale);
+      set_out16(ep, 1, g_lo + j * RP, 3 * RP, true, 1.0f, 0);
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+    }
+    for (int j = 0; j < 3; ++j) {
+      // dB_j = d{q,k,v}_pre^T u_j   [out_j, r]
+      lz.stage = ST_BWD_DB_QKV;
+      GemmCore core;
+      core_init(core, outj[j], RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], dqkv + col0[j], false, outj[j], M, nqkv) ||
+          !map2d_mn(&core.maps[2], u_qkv + j * RP, false, RP, M, 3 * RP))
+        return MOT_ERR_CUDA;
+      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, false, false, true, true), true, true);
+      core.num_segs = 1;
+      EpiStore::Params ep = store_params(outj[j], r);
+      ep.out32 = d_b[j];
+      ep.ld32 = r;
+      ep.accumulate32 = accumulate;
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+    }
+    for (int j = 0; j < 3; ++j) {
+      // dA_j = (s g_j)^T x   [r, d], computed as its transpose x^T (s g_j)_hi + x^T (s g_j)_lo
+      lz.stage = ST_BWD_DA_QKV;
+      GemmCore core;
+      core_init(core, d, RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], x, true, d, M, d) || !map2d_mn(&core.maps[2], g_hi + j * RP, true, RP, M, 3 * RP) ||
+          !map2d_mn(&core.maps[3], g_lo + j * RP, true, RP, M, 3 * RP))
+        return MOT_ERR_CUDA;
+      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
+      core.segs[1] = seg1(0, 0, 3, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
+      core.num_segs = 2;
+      EpiStore::Params ep = store_params(d, r);
+      ep.out32 = d_a[j];
+      ep.ld32 = d;
+      ep.accumulate32 = accumulate;
+      ep.transpose32 = 1;
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+    }
+  }
+  // dx = dq W_q + dk W_k + dv W_v + sum_j ((s g_j)_hi + (s g_j)_lo) A_j
+  lz.stage = ST_BWD_DX;
+  {
+    GemmCore core;
+    core_init(core, M, d, 256, 256, h->status);
+    bool ok = map2d(&core.maps[0], dqkv, false, nqkv, M, nqkv, 128);
+    if (r > 0)
+      ok = ok && map2d(&core.maps[1], g_hi, true, 3 * RP, M, 3 * RP, 128) &&
+           map2d(&core.maps[8], g_lo, true, 3 * RP, M, 3 * RP, 128);
+    if (!ok) return MOT_ERR_CUDA;
+    core.maps[2] = h->wq16_mn;
+    core.maps[3] = h->wk16_mn;
+    core.maps[4] = h->wv16_mn;
+    for (int j = 0; j < 3; ++j)
+      core.segs[j] = seg1(0, col0[j], 2 + j, outj[j] / 64, idesc_f16(128, 256, false, false, false, true), false, true);
+    core.num_segs = 3;
+    if (r > 0) {
+      core.maps[5] = h->aq_mn;
+      core.maps[6] = h->ak_mn;
+      core.maps[7] = h->av_mn;
+      for (int j = 0; j < 3; ++j) {
+        core.segs[3 + j] = seg1(1, j * RP, 5 + j, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+        core.segs[6 + j] = seg1(8, j * RP, 5 + j, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+      }
+      core.num_segs = 9;
+    }
+    EpiStore::Params ep = store_params(M, d);
+    set_out16(ep, 0, dx, d, true);
+    ep.out32 = dx_f32;
+    ep.ld32 = d;
+    lz.done(launch_gemm<256, 4, EpiStore>(core, ep, h->num_sms, st));
+  }
+  return lz.finish();
 }
 
 mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void* w_v_out, void* w_o_out,
@@ -576,7 +1010,7 @@ mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void*
         return MOT_ERR_CUDA;
   }
   if (cudaGetLastError() != cudaSuccess) return MOT_ERR_CUDA;
-  // rebind: merged base, no adapters; W_o's f16 copy is rebuilt from the merged W_o
+  // rebind: merged base, no adapters; the f16 copies are rebuilt from the merged weights
   h->w.w_q = w_q_out;
   h->w.w_k = w_k_out;
   h->w.w_v = w_v_out;
@@ -587,11 +1021,11 @@ mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void*
   h->RP = 0;
   h->scale = 0.f;
   h->cfg.lora_rank = 0;
-  bf16_to_f16_kernel<<<2 * h->num_sms, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w_o_out), h->wo16,
-                                                     static_cast<long long>(d) * qd / 8, h->status);
-  if (cudaGetLastError() != cudaSuccess) return MOT_ERR_CUDA;
+  if (refresh_f16_copies(h, st) != cudaSuccess) return MOT_ERR_CUDA;
   return build_weight_maps(h);
 }
+
+}  // extern "C"
 
 // ------------------------------------------------------------------ no-allocation forward
 // Scratch of mot_attn_forward_noalloc: one file-scope device array. In host
@@ -638,6 +1072,8 @@ extern "C" mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int3
 }
 
 // ------------------------------------------------------------------ dev entry points
+extern "C" {
+
 mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, int32_t n, int32_t k, int32_t is_bf16,
                         void* stream) {
   if (!a || !b || !dmat || m <= 0 || n <= 0 || k <= 0) return MOT_ERR_INVALID_ARGUMENT;
@@ -645,12 +1081,17 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, in
   if (!aligned16(a) || !aligned16(b) || !aligned16(dmat)) return MOT_ERR_ALIGNMENT;
   GemmCore core;
   const bool bf = is_bf16 != 0;
-  core_init(core, m, n, 256, k / 64, 0, 256, idesc_f16(128, 256, bf, bf), 0, nullptr);
+  core_init(core, m, n, 256, 256, nullptr);
   if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, 256)) return MOT_ERR_CUDA;
-  core.num_regions = 1;
-  core.regions[0] = GemmRegion{0, n, 2, -1, 0};
-  EpiStore::Params ep{nullptr, 0, 0, dmat, n, 0, 1.0f, m, n, 0};
-  return launch_gemm<256, 4, EpiStore>(core, ep, 148, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(128, 256, bf, bf), false, false);
+  core.num_segs = 1;
+  EpiStore::Params ep = store_params(m, n);
+  ep.out32 = dmat;
+  ep.ld32 = n;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return launch_gemm<256, 4, EpiStore>(core, ep, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOT_OK
              : MOT_ERR_CUDA;
 }
