@@ -126,6 +126,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     *abort_flag = 0u;
     fence_mbar_init();
   }
+  if (warp == 0 && lane == 0) {
+    // pull every tensor map the segments use into the descriptor cache
+    for (int si = 0; si < g.num_segs; ++si) {
+      tma_prefetch_desc(&g.maps[g.segs[si].a_map]);
+      for (int r = 0; r < g.num_regions; ++r) tma_prefetch_desc(&g.maps[g.segs[si].b_map[r]]);
+    }
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -138,42 +145,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
   const int num_tiles = g.tiles_m * g.tiles_n;
 
+  // Both issuing threads copy what they need out of the parameter block into
+  // registers before their K loops: the TMA / MMA wrappers clobber memory, so
+  // fields read through a reference would be re-fetched after every issue.
+  const int num_segs = g.num_segs;
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      const int b_box_rows = g.b_box_rows;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
         const int m0 = tm * kBM, n0 = tn * BN;
         const int reg0 = region_of(g, n0);
-        for (int si = 0; si < g.num_segs; ++si) {
+        for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
-          for (int kb = 0; kb < sg.kb; ++kb) {
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb, a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
+          const CUtensorMap* amap = &g.maps[sg.a_map];
+          // B boxes of this tile: up to 4 (map, row/column offset) pairs
+          const int box_n = b_mn ? 64 : b_box_rows;
+          const int nbox = BN / box_n;
+          const CUtensorMap* bmap[4];
+          int bcoord[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int n = n0 + (i < nbox ? i : 0) * box_n;
+            const int r = region_of(g, n);
+            bmap[i] = &g.maps[sg.b_map[r]];
+            bcoord[i] = n - g.region_n0[r];
+          }
+          const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
+          for (int kb = 0; kb < nkb; ++kb) {
             mbar_wait(&empty[stage], phase ^ 1u, wg);
             mbar_expect_tx(&full[stage], L::kABytes + L::kBBytes);
             uint8_t* a_dst = sA + stage * L::kABytes;
             uint8_t* b_dst = sB + stage * L::kBBytes;
-            const int ka = sg.a_k0[reg0] + kb * kBK, kbk = sg.b_k0 + kb * kBK;
-            if (sg.a_mn) {
-              tma_load_2d(a_dst, &g.maps[sg.a_map], &full[stage], m0, ka);
-              tma_load_2d(a_dst + kMnBoxBytes, &g.maps[sg.a_map], &full[stage], m0 + 64, ka);
+            const int ka = a_k0 + kb * kBK, kbk = b_k0 + kb * kBK;
+            if (a_mn) {
+              tma_load_2d(a_dst, amap, &full[stage], m0, ka);
+              tma_load_2d(a_dst + kMnBoxBytes, amap, &full[stage], m0 + 64, ka);
             } else {
-              tma_load_2d(a_dst, &g.maps[sg.a_map], &full[stage], ka, m0);
+              tma_load_2d(a_dst, amap, &full[stage], ka, m0);
             }
-            if (sg.b_mn) {
-              for (int i = 0; i < BN / 64; ++i) {
-                const int n = n0 + i * 64;
-                const int r = region_of(g, n);
-                tma_load_2d(b_dst + i * kMnBoxBytes, &g.maps[sg.b_map[r]], &full[stage], n - g.region_n0[r], kbk);
-              }
-            } else {
-              const uint32_t box_bytes = static_cast<uint32_t>(g.b_box_rows) * kBK * 2;
-              for (int i = 0; i < BN / g.b_box_rows; ++i) {
-                const int n = n0 + i * g.b_box_rows;
-                const int r = region_of(g, n);
-                tma_load_2d(b_dst + i * box_bytes, &g.maps[sg.b_map[r]], &full[stage], kbk, n - g.region_n0[r]);
-              }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (i >= nbox) break;
+              if (b_mn)
+                tma_load_2d(b_dst + i * box_bytes, bmap[i], &full[stage], bcoord[i], kbk);
+              else
+                tma_load_2d(b_dst + i * box_bytes, bmap[i], &full[stage], kbk, bcoord[i]);
             }
             if (++stage == STAGES) {
               stage = 0;
@@ -193,20 +214,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        bool first = true;
-        for (int si = 0; si < g.num_segs; ++si) {
+        uint32_t accumulate = 0u;
+        for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
-          for (int kb = 0; kb < sg.kb; ++kb) {
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb;
+          const uint32_t idesc = sg.idesc;
+          for (int kb = 0; kb < nkb; ++kb) {
             mbar_wait(&full[stage], phase, wg);
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
             const uint32_t b_addr = smem_u32(sB + stage * L::kBBytes);
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = sg.a_mn ? mnmajor_desc(a_addr, kk, kMnBoxBytes) : kmajor_desc(a_addr, kk, L::kABytes);
-              const uint64_t bd = sg.b_mn ? mnmajor_desc(b_addr, kk, kMnBoxBytes) : kmajor_desc(b_addr, kk, L::kBBytes);
-              umma_ss(d_tmem, ad, bd, sg.idesc, first ? 0u : 1u);
-              first = false;
+              const uint64_t ad = a_mn ? mnmajor_desc(a_addr, kk, kMnBoxBytes) : kmajor_desc(a_addr, kk, L::kABytes);
+              const uint64_t bd = b_mn ? mnmajor_desc(b_addr, kk, kMnBoxBytes) : kmajor_desc(b_addr, kk, L::kBBytes);
+              umma_ss(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1u;
             }
             umma_commit(&empty[stage]);
             if (++stage == STAGES) {
