@@ -458,9 +458,15 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
       const int h = g * G + it / p.q_tiles, qi = it % p.q_tiles;
       const long long sbase = (static_cast<long long>(b) * p.Hq + h) * p.N + qi * 128;
       const int qvalid = p.N - qi * 128;
-      // per-query softmax statistics of this tile (volatile: read in place, not hoisted)
-      const volatile float* lse_t = p.lse + sbase;
-      const volatile float* del_t = p.delta + sbase;
+      // softmax statistics of this tile's 128 queries: lane l holds queries
+      // l, l+32, l+64, l+96; column c is read from lane c%32 by a shuffle
+      float lse_r[4], del_r[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int q = lane + 32 * k;
+        lse_r[k] = q < qvalid ? p.lse[sbase + q] * kLog2e : 0.f;
+        del_r[k] = q < qvalid ? p.delta[sbase + q] : 0.f;
+      }
       mbar_wait(sdp_full, it & 1, wg);
       tc_fence_after();
       // the A buffer holds dScore^T of the previous iteration until its dK MMA is done
@@ -477,10 +483,10 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
         for (int i = 0; i < 16; i += 2) {
           const int col = c * 16 + i;
           const bool v0 = col < qvalid, v1 = col + 1 < qvalid;
-          const float l0 = v0 ? lse_t[col] * kLog2e : 0.f;
-          const float l1 = v1 ? lse_t[col + 1] * kLog2e : 0.f;
-          const float D0 = v0 ? del_t[col] : 0.f;
-          const float D1 = v1 ? del_t[col + 1] : 0.f;
+          const float l0 = __shfl_sync(0xffffffffu, lse_r[col >> 5], col & 31);
+          const float l1 = __shfl_sync(0xffffffffu, lse_r[(col + 1) >> 5], (col + 1) & 31);
+          const float D0 = __shfl_sync(0xffffffffu, del_r[col >> 5], col & 31);
+          const float D1 = __shfl_sync(0xffffffffu, del_r[(col + 1) >> 5], (col + 1) & 31);
           float p0 = ex2_approx(fmaf(__uint_as_float(rs[i]), p.scale_log2, -l0));
           float p1 = ex2_approx(fmaf(__uint_as_float(rs[i + 1]), p.scale_log2, -l1));
           p0 = v0 ? p0 : 0.f;

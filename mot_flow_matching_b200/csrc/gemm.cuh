@@ -402,6 +402,38 @@ struct EpiStore {
   }
 };
 
+// LoRA gradients of q, k and v from one GEMM whose N columns are three
+// rank-wide blocks (block j = columns [j*RP, (j+1)*RP), of which the first r
+// are real): block j is added into (or written to) out[j], transposed
+// (element (m, k) at out[j][k * ld + m]) or not (at out[j][m * ld + k]).
+struct EpiLoraGrad {
+  struct Params {
+    float* out[3];
+    long long ld;
+    int RP, r, M;
+    int transpose, accumulate;
+  };
+  template <int BN>
+  __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
+                                               int* status) {
+    const int m = m0 + row;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      load_row32(taddr + c, v);
+      if (m >= p.M) continue;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int n = n0 + c + i;
+        const int j = n / p.RP, k = n - j * p.RP;
+        if (j > 2 || k >= p.r) continue;
+        float* o = p.transpose ? p.out[j] + static_cast<long long>(k) * p.ld + m : p.out[j] + m * p.ld + k;
+        *o = p.accumulate ? *o + v[i] : v[i];
+      }
+    }
+  }
+};
+
 // Gradient of the attention output: stores dO = acc as f16 [M, Hq*dh] and,
 // per (token, head), D = sum_j dO_j O_j with the forward's attention output O
 // (the rowsum the softmax backward subtracts), taken over the f16-rounded dO

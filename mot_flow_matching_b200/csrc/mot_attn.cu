@@ -891,19 +891,28 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     lz.done(cudaGetLastError());
   }
   if (r > 0) {
-    for (int j = 0; j < 3; ++j) {
-      // g_j = d{q,k,v}_pre B_j  -> s g_j as bf16 hi + lo in columns [j*RP, (j+1)*RP)
+    {
+      // g_j = d{q,k,v}_pre B_j for the three projections in one GEMM: column
+      // block j reads its own K range of d{q,k,v}_pre (B_k, B_v are zero past
+      // their rows) -> s g_j as bf16 hi + lo in columns [j*RP, (j+1)*RP)
       lz.stage = ST_BWD_G_QKV;
       GemmCore core;
-      core_init(core, M, RP, RP, RP, h->status);
-      if (!map2d(&core.maps[0], dqkv, false, nqkv, M, nqkv, 128) ||
-          !map2d_mn(&core.maps[2], b16 + static_cast<long long>(col0[j]) * r, false, r, outj[j], r))
-        return MOT_ERR_CUDA;
-      core.segs[0] = seg1(0, col0[j], 2, outj[j] / 64, idesc_f16(128, RP, false, false, false, true), false, true);
+      core_init(core, M, 3 * RP, RP, RP, h->status);
+      if (!map2d(&core.maps[0], dqkv, false, nqkv, M, nqkv, 128)) return MOT_ERR_CUDA;
+      for (int j = 0; j < 3; ++j)
+        if (!map2d_mn(&core.maps[2 + j], b16 + static_cast<long long>(col0[j]) * r, false, r, outj[j], r))
+          return MOT_ERR_CUDA;
+      core.num_regions = 3;
+      for (int j = 0; j <= 3; ++j) core.region_n0[j] = j * RP;
+      core.segs[0] = seg1(0, 0, 2, qd / 64, idesc_f16(128, RP, false, false, false, true), false, true);
+      for (int j = 0; j < 3; ++j) {
+        core.segs[0].a_k0[j] = col0[j];
+        core.segs[0].b_map[j] = 2 + j;
+      }
       core.num_segs = 1;
-      EpiStore::Params ep = store_params(M, RP);
-      set_out16(ep, 0, g_hi + j * RP, 3 * RP, true, h->scale);
-      set_out16(ep, 1, g_lo + j * RP, 3 * RP, true, 1.0f, 0);
+      EpiStore::Params ep = store_params(M, 3 * RP);
+      set_out16(ep, 0, g_hi, 3 * RP, true, h->scale);
+      set_out16(ep, 1, g_lo, 3 * RP, true, 1.0f, 0);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
     for (int j = 0; j < 3; ++j) {
@@ -922,23 +931,27 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.accumulate32 = accumulate;
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
-    for (int j = 0; j < 3; ++j) {
-      // dA_j = (s g_j)^T x   [r, d], computed as its transpose x^T (s g_j)_hi + x^T (s g_j)_lo
+    {
+      // dA_j = (s g_j)^T x for the three projections in one GEMM over x^T,
+      // with (s g_j) as its bf16 hi + lo pair; block j goes to dA_j transposed
       lz.stage = ST_BWD_DA_QKV;
       GemmCore core;
-      core_init(core, d, RP, RP, RP, h->status);
-      if (!map2d_mn(&core.maps[0], x, true, d, M, d) || !map2d_mn(&core.maps[2], g_hi + j * RP, true, RP, M, 3 * RP) ||
-          !map2d_mn(&core.maps[3], g_lo + j * RP, true, RP, M, 3 * RP))
+      core_init(core, d, 3 * RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], x, true, d, M, d) || !map2d_mn(&core.maps[2], g_hi, true, 3 * RP, M, 3 * RP) ||
+          !map2d_mn(&core.maps[3], g_lo, true, 3 * RP, M, 3 * RP))
         return MOT_ERR_CUDA;
       core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
       core.segs[1] = seg1(0, 0, 3, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
       core.num_segs = 2;
-      EpiStore::Params ep = store_params(d, r);
-      ep.out32 = d_a[j];
-      ep.ld32 = d;
-      ep.accumulate32 = accumulate;
-      ep.transpose32 = 1;
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+      EpiLoraGrad::Params ep{};
+      for (int j = 0; j < 3; ++j) ep.out[j] = d_a[j];
+      ep.ld = d;
+      ep.RP = RP;
+      ep.r = r;
+      ep.M = d;
+      ep.transpose = 1;
+      ep.accumulate = accumulate;
+      lz.done(launch_gemm_narrow<EpiLoraGrad>(RP, core, ep, h->num_sms, st));
     }
   }
   // dx = dq W_q + dk W_k + dv W_v + sum_j ((s g_j)_hi + (s g_j)_lo) A_j
