@@ -1,38 +1,42 @@
 // attn_fwd.cuh -- grouped-query attention forward over [prefix cache ; self]
 // on sm_100a tensor cores.
 //
-// For one CFG branch b, query head h and a 128-row tile of image tokens:
+// For one CFG branch b, query head h and image tokens i:
 //   o = softmax(q^ K^T / sqrt(dh)) V,  K, V = rows [0, prefix_len[b] + N) of the
 //   KV head g = h / (Hq/Hkv) ("SenseNova-U1" DiffSynth-Studio docs,
 //   architecture note: image tokens attend to the prefix cache; vLLM-Omni
 //   "SenseNova-U1" recipe, kernel table: "dual-tower attention" in a flash
 //   kernel). Non-causal; keys past prefix_len[b] + N are masked.
 //
-// Per CTA: warp 0 streams Q once and K/V tiles (128 keys x 128 dims, f16,
-// 128-byte swizzle) by TMA into a 2-deep ring; warp 1 issues
-//   S_j = Q K_j^T   into one of two TMEM buffers (M=128, N=128, K=16 x 8)
-//   O  += P_j V_j   into a TMEM accumulator (V is the MN-major operand)
-// in the order S0, S1, PV0, S2, PV1, ... so the tensor core computes S_{j+1}
-// while warps 2..5 (one query row per thread) turn S_j into P_j:
-// running max m and sum l in fp32, p = 2^(s*log2(e)/sqrt(dh) - m) written as
-// f16 into a swizzled K-major smem tile. The running max is only raised
-// (and O rescaled through TMEM) when a row's max grows by more than 2^8, so
-// p <= 256 stays exact enough in f16 and the final o = O / l uses the same m
-// as every p it summed: the result is unchanged by the laziness.
+// One CTA owns two 128-query tiles (t = 0, 1) of one (b, h) and streams the
+// key/value tiles (128 keys x 128 dims, f16, 128-byte swizzle) once for both
+// through a 2-deep TMA ring. TMEM holds, per query tile, S_t (128 f32
+// columns) and the output accumulator O_t (128 columns). Warp 1 issues, per
+// key tile j,
+//   S_0 = Q_0 K_j^T, S_1 = Q_1 K_j^T, then O_0 += P_0 V_j, S_0 <- next tile,
+//   O_1 += P_1 V_j, S_1 <- next tile
+// so the tensor core works on one query tile while the other's softmax runs.
+// Warps 2-5 (tile 0) and 6-9 (tile 1) hold one query row per thread: they
+// read S_t from TMEM, keep the running max m and sum l in f32, and write
+// p = 2^(s log2(e)/sqrt(dh) - m) as f16 pairs back over the first 64 columns
+// of S_t, where the P V MMA reads it as its TMEM operand (no shared-memory
+// round trip). The running max is only raised, and O_t rescaled through
+// TMEM, when a row's max grows by more than 2^8; p <= 256 is exact enough in
+// f16 and the final o = O / l uses the same m as every p it summed.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace mot {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
 constexpr float kLazyRescaleLog2 = 8.0f;
 
 struct AttnFwdParams {
   CUtensorMap q_map;  // 3D {dh, N, B*Hq} f16, box {64, 128, 1}
   CUtensorMap k_map;  // 3D {dh, Lcap, B*Hkv} f16, box {64, 128, 1}
   CUtensorMap v_map;  // same as k_map
-  int B, N, Hq, Hkv, Lcap, q_tiles;
+  int B, N, Hq, Hkv, Lcap, q_pairs;  // q_pairs = ceil(N / 256)
   int plen[kMaxBatch];
   float scale_log2;  // log2(e) / sqrt(dh)
   __half* out;       // [B*N, Hq*dh] token-major
@@ -42,39 +46,86 @@ struct AttnFwdParams {
 
 struct AttnSmem {
   static constexpr uint32_t kTile = 32768;  // 128 rows x 128 f16
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTile;
+  static constexpr uint32_t kQ = 0;         // two query tiles
+  static constexpr uint32_t kK = kQ + 2 * kTile;
   static constexpr uint32_t kV = kK + 2 * kTile;
-  static constexpr uint32_t kP = kV + 2 * kTile;
-  static constexpr uint32_t kBar = kP + 2 * kTile;
+  static constexpr uint32_t kBar = kV + 2 * kTile;
   static constexpr uint32_t kBytes = kBar + 256 + 1024;
 };
+
+// max over 128 scores in four independent chains (columns >= valid masked to -inf)
+template <bool kFull>
+__device__ __forceinline__ float tile_row_max(uint32_t taddr, int valid) {
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = (kFull || c * 32 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
+      mx[i & 3] = fmaxf(mx[i & 3], v);
+    }
+  }
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// p = 2^(s c - m) for the 128 scores of this row, written as f16 pairs over
+// the first 64 columns of S (chunk c of P covers S columns [32c, 32c+32),
+// already read when it is written); returns the row sum of p.
+template <bool kFull>
+__device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float scale, float neg_m) {
+  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      float x0, x1;
+      ffma2(x0, x1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), scale, scale, neg_m, neg_m);
+      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      if (!kFull) {
+        p0 = c * 32 + i < valid ? p0 : 0.f;
+        p1 = c * 32 + i + 1 < valid ? p1 : 0.f;
+      }
+      if ((i >> 1) & 1)
+        fadd2(sc, sd, sc, sd, p0, p1);
+      else
+        fadd2(sa, sb, sa, sb, p0, p1);
+      pk[i >> 1] = pack_half2(p0, p1);
+    }
+    tmem_st16(taddr + c * 16, pk);
+  }
+  return (sa + sb) + (sc + sd);
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t T32 = AttnSmem::kTile;
   uint8_t* sQ = smem + AttnSmem::kQ;
   uint8_t* sK = smem + AttnSmem::kK;
   uint8_t* sV = smem + AttnSmem::kV;
-  uint8_t* sP = smem + AttnSmem::kP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_full = bars + 1;    // [2] ring stages
   uint64_t* k_empty = bars + 3;   // [2]
   uint64_t* v_full = bars + 5;    // [2]
   uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* s_free = bars + 11;   // [2]
-  uint64_t* p_full = bars + 13;   // [2]
-  uint64_t* p_free = bars + 15;   // [2]
-  uint64_t* o_full = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* s_full = bars + 9;    // [2] query tiles
+  uint64_t* p_full = bars + 11;   // [2]
+  uint64_t* o_done = bars + 13;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = warp_id(), lane = lane_id();
   int bid = blockIdx.x;
-  const int qt = bid % p.q_tiles;
-  bid /= p.q_tiles;
+  const int qp = bid % p.q_pairs;
+  bid /= p.q_pairs;
   const int h = bid % p.Hq;
   const int b = bid / p.Hq;
   const int g = h / (p.Hq / p.Hkv);
@@ -89,11 +140,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
-      mbar_init(&p_free[i], 1);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(o_full, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -104,8 +153,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tO = tmem_base + 256u;
+  const uint32_t tmem = *tmem_slot;
   const WaitGuard wg{abort_flag, p.status};
 
   if (warp == 0) {
@@ -114,93 +162,87 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       tma_prefetch_desc(&p.k_map);
       tma_prefetch_desc(&p.v_map);
       const int qz = b * p.Hq + h, kz = b * p.Hkv + g;
-      mbar_expect_tx(q_full, AttnSmem::kTile);
-      tma_load_3d(sQ, &p.q_map, q_full, 0, qt * 128, qz);
-      tma_load_3d(sQ + 16384, &p.q_map, q_full, 64, qt * 128, qz);
+      mbar_expect_tx(q_full, 2 * T32);
+      for (int t = 0; t < 2; ++t) {
+        tma_load_3d(sQ + t * T32, &p.q_map, q_full, 0, qp * 256 + t * 128, qz);
+        tma_load_3d(sQ + t * T32 + 16384, &p.q_map, q_full, 64, qp * 256 + t * 128, qz);
+      }
       for (int j = 0; j < T; ++j) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         mbar_wait(&k_empty[s], ph ^ 1u, wg);
-        mbar_expect_tx(&k_full[s], AttnSmem::kTile);
-        tma_load_3d(sK + s * AttnSmem::kTile, &p.k_map, &k_full[s], 0, j * 128, kz);
-        tma_load_3d(sK + s * AttnSmem::kTile + 16384, &p.k_map, &k_full[s], 64, j * 128, kz);
+        mbar_expect_tx(&k_full[s], T32);
+        tma_load_3d(sK + s * T32, &p.k_map, &k_full[s], 0, j * 128, kz);
+        tma_load_3d(sK + s * T32 + 16384, &p.k_map, &k_full[s], 64, j * 128, kz);
         mbar_wait(&v_empty[s], ph ^ 1u, wg);
-        mbar_expect_tx(&v_full[s], AttnSmem::kTile);
-        tma_load_3d(sV + s * AttnSmem::kTile, &p.v_map, &v_full[s], 0, j * 128, kz);
-        tma_load_3d(sV + s * AttnSmem::kTile + 16384, &p.v_map, &v_full[s], 64, j * 128, kz);
+        mbar_expect_tx(&v_full[s], T32);
+        tma_load_3d(sV + s * T32, &p.v_map, &v_full[s], 0, j * 128, kz);
+        tma_load_3d(sV + s * T32 + 16384, &p.v_map, &v_full[s], 64, j * 128, kz);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16(128, 128, false, false, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(128, 128, false, false, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t q_addr[2] = {smem_u32(sQ), smem_u32(sQ + T32)};
+      auto issue_s = [&](int t, int j) {
+        const uint32_t k_addr = smem_u32(sK + (j & 1) * T32);
+        const uint32_t qa = t ? q_addr[1] : q_addr[0];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + t * 128u, kmajor_desc(qa, kk, 16384), kmajor_desc(k_addr, kk, 16384), idesc_qk, kk > 0);
+        umma_commit(&s_full[t]);
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t va = smem_u32(sV + (j & 1) * T32);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + 256u + t * 128u, tmem + t * 128u + kk * 8u, mnmajor_desc(va, kk, 16384), idesc_pv,
+                  (j | kk) != 0);
+        umma_commit(&o_done[t]);
+      };
       mbar_wait(q_full, 0, wg);
-      for (int j = 0; j <= T; ++j) {
-        if (j < T) {
-          const int s = j & 1;
-          mbar_wait(&k_full[s], (j >> 1) & 1, wg);
-          if (j >= 2) mbar_wait(&s_free[s], ((j - 2) >> 1) & 1, wg);
+      mbar_wait(&k_full[0], 0, wg);
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      umma_commit(&k_empty[0]);
+      for (int j = 0; j < T; ++j) {
+        const int s = j & 1;
+        const bool more = j + 1 < T;
+        mbar_wait(&v_full[s], (j >> 1) & 1, wg);
+        mbar_wait(&p_full[0], j & 1, wg);
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, wg);
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + s * AttnSmem::kTile);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tmem_base + static_cast<uint32_t>(s) * 128u, kmajor_desc(q_addr, kk, 16384), kmajor_desc(k_addr, kk, 16384), idesc_qk, kk > 0);
-          umma_commit(&s_full[s]);
-          umma_commit(&k_empty[s]);
+          issue_s(0, j + 1);  // overwrites P_0 only after the P V MMA above (in-order issue)
         }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj & 1;
-          const uint32_t ph = (jj >> 1) & 1;
-          mbar_wait(&p_full[s], ph, wg);
-          mbar_wait(&v_full[s], ph, wg);
-          tc_fence_after();
-          const uint32_t pa = smem_u32(sP + s * AttnSmem::kTile);
-          const uint32_t va = smem_u32(sV + s * AttnSmem::kTile);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tO, kmajor_desc(pa, kk, 16384), mnmajor_desc(va, kk, 16384), idesc_pv, (jj | kk) != 0);
-          umma_commit(&v_empty[s]);
-          umma_commit(&p_free[s]);
+        mbar_wait(&p_full[1], j & 1, wg);
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&v_empty[s]);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&k_empty[(j + 1) & 1]);
         }
       }
-      umma_commit(o_full);
     }
   } else {
-    const int quarter = warp & 3;
+    const int t = (warp - 2) >> 2;       // query tile of this warpgroup
+    const int quarter = warp & 3;        // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + t * 128u + lane_off;
+    const uint32_t tO = tmem + 256u + t * 128u + lane_off;
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < T; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      mbar_wait(&s_full[s], ph, wg);
+      mbar_wait(&s_full[t], j & 1, wg);
       tc_fence_after();
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + static_cast<uint32_t>(s) * 128u + lane_off + c * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[s]);
-
       const int valid = L - j * 128;  // keys of this tile that exist (>= 1)
-      float mx = -INFINITY;
-      if (valid >= 128) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          if (i >= valid) sv[i] = -INFINITY;
-          mx = fmaxf(mx, sv[i]);
-        }
-      }
-      const float m_tile = mx * p.scale_log2;
+      const bool full = valid >= 128;
+      const float m_tile = (full ? tile_row_max<true>(tS, valid) : tile_row_max<false>(tS, valid)) * p.scale_log2;
       bool need = false;
       float m_new = m_run;
       if (j == 0) {
@@ -209,61 +251,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         need = true;
         m_new = m_tile;
       }
-      // the P buffer this tile writes was last read by PV_{j-2}
-      if (j >= 2) mbar_wait(&p_free[s], ((j - 2) >> 1) & 1, wg);
-      if (__any_sync(0xffffffffu, need)) {
-        // O must be final up to PV_{j-1} before it is rescaled
-        mbar_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, wg);
+      // o_done completes once per P V of this tile; waiting on every phase in
+      // order keeps the parity unambiguous. S_t of this tile was issued after
+      // the previous P V, so that P V is already complete here: O is stable.
+      if (j >= 1) {
+        mbar_wait(&o_done[t], (j - 1) & 1, wg);
         tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
-          tmem_ld32(tO + lane_off + c * 32, r);
+          tmem_ld32(tO + c * 32, r);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + lane_off + c * 32, r);
+          tmem_st32(tO + c * 32, r);
         }
         tmem_st_wait();
         l_run *= alpha;
       }
       m_run = m_new;
-      float rowsum = 0.f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        sv[i] = ex2_approx(fmaf(sv[i], p.scale_log2, -m_run));
-        rowsum += sv[i];
-      }
-      l_run += rowsum;
-      uint8_t* pb = sP + s * AttnSmem::kTile + row * 128;
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 w;
-          const float* q = sv + hf * 64 + c * 8;
-          w.x = pack_half2(q[0], q[1]);
-          w.y = pack_half2(q[2], q[3]);
-          w.z = pack_half2(q[4], q[5]);
-          w.w = pack_half2(q[6], q[7]);
-          *reinterpret_cast<uint4*>(pb + hf * 16384 + ((c ^ (row & 7)) << 4)) = w;
-        }
-      }
-      fence_proxy_async_smem();
+      const float row_sum = full ? tile_row_exp<true>(tS, valid, p.scale_log2, -m_run)
+                                 : tile_row_exp<false>(tS, valid, p.scale_log2, -m_run);
+      tmem_st_wait();
+      l_run += row_sum;
       tc_fence_before();
-      mbar_arrive(&p_full[s]);
+      mbar_arrive(&p_full[t]);
     }
     // epilogue: o = O / l, token-major f16
-    mbar_wait(o_full, 0, wg);
+    mbar_wait(&o_done[t], (T - 1) & 1, wg);
     tc_fence_after();
-    const int qrow = qt * 128 + row;
+    const int qrow = qp * 256 + t * 128 + row;
     const float inv_l = 1.0f / l_run;
     __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t r[32];
-      tmem_ld32(tO + lane_off + c * 32, r);
+      tmem_ld32(tO + c * 32, r);
       tmem_ld_wait();
       if (qrow < p.N) {
         uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
@@ -285,7 +311,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -656,7 +656,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ap.Hq = Hq;
     ap.Hkv = Hkv;
     ap.Lcap = L.Lcap;
-    ap.q_tiles = (N + 127) / 128;
+    ap.q_pairs = (N + 255) / 256;
     for (int b = 0; b < B; ++b) ap.plen[b] = prefix_len[b];
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
     ap.out = attn;
@@ -664,7 +664,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ap.status = h->status;
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(attn_fwd_kernel, AttnSmem::kBytes); });
-    attn_fwd_kernel<<<B * Hq * ap.q_tiles, kAttnThreads, AttnSmem::kBytes, st>>>(ap);
+    attn_fwd_kernel<<<B * Hq * ap.q_pairs, kAttnThreads, AttnSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
   }
   // 6. LoRA down for o: u_o = s o A_o^T (f16; training also keeps it as a bf16 hi + lo pair)
