@@ -47,6 +47,11 @@ mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32
 mot_status mot_dev_profile(mot_attn_t h, int32_t enable);
 mot_status mot_dev_stage_times(mot_attn_t h, int32_t* ids, float* ms, int32_t max, int32_t* count);
 
+/* y[i] = 2^x[i] through the FMA-pipe exponential the attention softmax uses
+ * for part of its probabilities (range reduction + degree-3 polynomial);
+ * x, y device f32 [n], n even, x in [-125, 8]. For accuracy tests. */
+mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream);
+
 /* Static name of a stage id ("qkv_gemm", "attn_fwd", ...; "?" if unknown). */
 const char* mot_dev_stage_name(int32_t id);
 

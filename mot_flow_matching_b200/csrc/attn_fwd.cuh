@@ -63,9 +63,10 @@ __device__ __forceinline__ float tile_row_max(uint32_t taddr, int valid) {
     tmem_ld32(taddr + c * 32, r);
     tmem_ld_wait();
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float v = (kFull || c * 32 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
-      mx[i & 3] = fmaxf(mx[i & 3], v);
+    for (int i = 0; i < 32; i += 2) {
+      const float v0 = (kFull || c * 32 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
+      const float v1 = (kFull || c * 32 + i + 1 < valid) ? __uint_as_float(r[i + 1]) : -INFINITY;
+      mx[(i >> 1) & 3] = fmax3(mx[(i >> 1) & 3], v0, v1);
     }
   }
   return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
@@ -73,7 +74,8 @@ __device__ __forceinline__ float tile_row_max(uint32_t taddr, int valid) {
 
 // p = 2^(s c - m) for the 128 scores of this row, written as f16 pairs over
 // the first 64 columns of S (chunk c of P covers S columns [32c, 32c+32),
-// already read when it is written); returns the row sum of p.
+// already read when it is written); returns the row sum of p. Masked keys
+// (x = -inf) are zeroed after the exponential.
 template <bool kFull>
 __device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float scale, float neg_m) {
   float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
@@ -87,7 +89,15 @@ __device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float s
     for (int i = 0; i < 32; i += 2) {
       float x0, x1;
       ffma2(x0, x1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), scale, scale, neg_m, neg_m);
-      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      // one pair in four on the FMA pipe: the MUFU would otherwise need as
+      // long per tile as the tile's MMAs
+      float p0, p1;
+      if (((i >> 1) & 3) == 3) {
+        exp2_poly2(p0, p1, x0, x1);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
       if (!kFull) {
         p0 = c * 32 + i < valid ? p0 : 0.f;
         p1 = c * 32 + i + 1 < valid ? p1 : 0.f;

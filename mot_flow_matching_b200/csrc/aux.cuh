@@ -119,6 +119,12 @@ __global__ void __launch_bounds__(256) cvt_multi_kernel(const CvtJobs jobs, int*
   if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
 }
 
+// 2^x of a buffer through exp2_poly2 (accuracy tests of the softmax's FMA-pipe exponential)
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int npairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < npairs) exp2_poly2(y[2 * i], y[2 * i + 1], x[2 * i], x[2 * i + 1]);
+}
+
 // f32 copy of a bf16 vector (norm gains)
 __global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

@@ -1109,6 +1109,12 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, in
              : MOT_ERR_CUDA;
 }
 
+mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream) {
+  if (!x || !y || n <= 0 || (n & 1)) return MOT_ERR_INVALID_ARGUMENT;
+  exp2_poly_kernel<<<(n / 2 + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n / 2);
+  return cudaGetLastError() == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+}
+
 mot_status mot_dev_profile(mot_attn_t h, int32_t enable) {
   if (!h) return MOT_ERR_INVALID_ARGUMENT;
   if (enable && !h->ev[0])

@@ -122,6 +122,10 @@ def mot_dev_saved_layout(cfg: MotAttnConfig, batch, img_tokens, prefix_max):
     return list(offs), lcap.value
 
 
+def mot_dev_exp2_poly(x, y, stream=None) -> None:
+    check(lib().mot_dev_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "mot_dev_exp2_poly")
+
+
 def mot_dev_profile(h, enable: bool) -> None:
     check(lib().mot_dev_profile(h, int(bool(enable))), "mot_dev_profile")
 
