@@ -16,8 +16,10 @@
 //   S_0 = Q_0 K_j^T, S_1 = Q_1 K_j^T, then O_0 += P_0 V_j, S_0 <- next tile,
 //   O_1 += P_1 V_j, S_1 <- next tile
 // so the tensor core works on one query tile while the other's softmax runs.
-// Warps 2-5 (tile 0) and 6-9 (tile 1) hold one query row per thread: they
-// read S_t from TMEM, keep the running max m and sum l in f32, and write
+// Warps 2-9 (tile 0) and 10-17 (tile 1) run the softmax, two threads per
+// query row, 64 score columns each (the halves swap partial maxima through
+// shared memory at a named barrier of the tile's 256 threads): they read S_t
+// from TMEM, keep the running max m and sum l in f32, and write
 // p = 2^(s log2(e)/sqrt(dh) - m) as f16 pairs back over the first 64 columns
 // of S_t, where the P V MMA reads it as its TMEM operand (no shared-memory
 // round trip). The running max is only raised, and O_t rescaled through
@@ -29,7 +31,7 @@
 
 namespace mot {
 
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 576;  // TMA warp, MMA warp, 2 x 8 softmax warps
 constexpr float kLazyRescaleLog2 = 8.0f;
 
 struct AttnFwdParams {
@@ -49,48 +51,55 @@ struct AttnSmem {
   static constexpr uint32_t kQ = 0;         // two query tiles
   static constexpr uint32_t kK = kQ + 2 * kTile;
   static constexpr uint32_t kV = kK + 2 * kTile;
-  static constexpr uint32_t kBar = kV + 2 * kTile;
+  static constexpr uint32_t kXch = kV + 2 * kTile;  // [2 tiles][2 buffers][2 halves][128] f32
+  static constexpr uint32_t kBar = kXch + 4096;
   static constexpr uint32_t kBytes = kBar + 256 + 1024;
 };
 
-// max over 128 scores in four independent chains (columns >= valid masked to -inf)
+// Half a row of S (64 f32 scores) in registers: two TMEM loads, one wait.
+struct HalfRowS {
+  uint32_t r[2][32];
+};
+
+__device__ __forceinline__ void load_half_row(uint32_t taddr, HalfRowS& s) {
+  tmem_ld32(taddr, s.r[0]);
+  tmem_ld32(taddr + 32, s.r[1]);
+  tmem_ld_wait();
+}
+
+// max over this thread's 64 scores (columns col0 + [0, 64); >= valid masked)
 template <bool kFull>
-__device__ __forceinline__ float tile_row_max(uint32_t taddr, int valid) {
+__device__ __forceinline__ float half_row_max(const HalfRowS& s, int col0, int valid) {
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
-    tmem_ld_wait();
+  for (int c = 0; c < 2; ++c) {
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
-      const float v0 = (kFull || c * 32 + i < valid) ? __uint_as_float(r[i]) : -INFINITY;
-      const float v1 = (kFull || c * 32 + i + 1 < valid) ? __uint_as_float(r[i + 1]) : -INFINITY;
+      const int col = col0 + c * 32 + i;
+      const float v0 = (kFull || col < valid) ? __uint_as_float(s.r[c][i]) : -INFINITY;
+      const float v1 = (kFull || col + 1 < valid) ? __uint_as_float(s.r[c][i + 1]) : -INFINITY;
       mx[(i >> 1) & 3] = fmax3(mx[(i >> 1) & 3], v0, v1);
     }
   }
   return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// p = 2^(s c - m) for the 128 scores of this row, written as f16 pairs over
-// the first 64 columns of S (chunk c of P covers S columns [32c, 32c+32),
-// already read when it is written); returns the row sum of p. Masked keys
-// (x = -inf) are zeroed after the exponential.
+// p = 2^(s c - m) for this thread's 64 scores, written as 32 f16 pairs at P
+// columns [col0/2, col0/2 + 32) of S; returns their sum. Masked keys are
+// zeroed after the exponential. One pair in four goes through the FMA-pipe
+// exponential, the rest through the MUFU.
 template <bool kFull>
-__device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float scale, float neg_m) {
+__device__ __forceinline__ float half_row_exp_store(const HalfRowS& s, uint32_t taddr_p, int col0, int valid,
+                                                    float scale, float neg_m) {
   float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
-    tmem_ld_wait();
+  for (int c = 0; c < 2; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
+      const int col = col0 + c * 32 + i;
       float x0, x1;
-      ffma2(x0, x1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), scale, scale, neg_m, neg_m);
-      // one pair in four on the FMA pipe: the MUFU would otherwise need as
-      // long per tile as the tile's MMAs
+      ffma2(x0, x1, __uint_as_float(s.r[c][i]), __uint_as_float(s.r[c][i + 1]), scale, scale, neg_m, neg_m);
       float p0, p1;
       if (((i >> 1) & 3) == 3) {
         exp2_poly2(p0, p1, x0, x1);
@@ -99,8 +108,8 @@ __device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float s
         p1 = ex2_approx(x1);
       }
       if (!kFull) {
-        p0 = c * 32 + i < valid ? p0 : 0.f;
-        p1 = c * 32 + i + 1 < valid ? p1 : 0.f;
+        p0 = col < valid ? p0 : 0.f;
+        p1 = col + 1 < valid ? p1 : 0.f;
       }
       if ((i >> 1) & 1)
         fadd2(sc, sd, sc, sd, p0, p1);
@@ -108,9 +117,13 @@ __device__ __forceinline__ float tile_row_exp(uint32_t taddr, int valid, float s
         fadd2(sa, sb, sa, sb, p0, p1);
       pk[i >> 1] = pack_half2(p0, p1);
     }
-    tmem_st16(taddr + c * 16, pk);
+    tmem_st16(taddr_p + c * 16, pk);
   }
   return (sa + sb) + (sc + sd);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnFwdParams p) {
@@ -150,7 +163,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
       mbar_init(&o_done[i], 1);
     }
     *abort_flag = 0u;
@@ -240,19 +253,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
     }
   } else {
-    const int t = (warp - 2) >> 2;       // query tile of this warpgroup
-    const int quarter = warp & 3;        // TMEM lane quarter this warp may access
+    const int t = (warp - 2) >> 3;           // query tile of these 8 warps
+    const int half = ((warp - 2) >> 2) & 1;  // score columns [64 half, 64 half + 64)
+    const int quarter = warp & 3;            // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
+    const int col0 = half * 64;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + t * 128u + lane_off;
     const uint32_t tO = tmem + 256u + t * 128u + lane_off;
-    float m_run = -INFINITY, l_run = 0.f;
+    float* xch = reinterpret_cast<float*>(smem + AttnSmem::kXch) + t * 512;  // [2 buffers][2 halves][128]
+    const int bar_id = 1 + t;
+    float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's partial row sum
     for (int j = 0; j < T; ++j) {
       mbar_wait(&s_full[t], j & 1, wg);
       tc_fence_after();
       const int valid = L - j * 128;  // keys of this tile that exist (>= 1)
       const bool full = valid >= 128;
-      const float m_tile = (full ? tile_row_max<true>(tS, valid) : tile_row_max<false>(tS, valid)) * p.scale_log2;
+      HalfRowS srow;
+      load_half_row(tS + col0, srow);
+      const float pm = full ? half_row_max<true>(srow, col0, valid) : half_row_max<false>(srow, col0, valid);
+      float* xb = xch + (j & 1) * 256;
+      xb[half * 128 + row] = pm;
+      // both halves hold their scores in registers past this barrier, so P
+      // may overwrite S; the partial maxima are exchanged through smem
+      named_bar_sync(bar_id, 256);
+      const float m_tile = fmaxf(pm, xb[(half ^ 1) * 128 + row]) * p.scale_log2;
       bool need = false;
       float m_new = m_run;
       if (j == 0) {
@@ -268,38 +293,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         mbar_wait(&o_done[t], (j - 1) & 1, wg);
         tc_fence_after();
       }
+      const float m_old = m_run;
+      m_run = m_new;
+      const float part = full ? half_row_exp_store<true>(srow, tS + half * 32, col0, valid, p.scale_log2, -m_run)
+                              : half_row_exp_store<false>(srow, tS + half * 32, col0, valid, p.scale_log2, -m_run);
+      // this half's O columns move to the new max (the next P V waits for p_full)
       if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+        const float alpha = need ? ex2_approx(m_old - m_new) : 1.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
+          tmem_ld32(tO + col0 + c * 32, r);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + c * 32, r);
+          tmem_st32(tO + col0 + c * 32, r);
         }
-        tmem_st_wait();
         l_run *= alpha;
       }
-      m_run = m_new;
-      const float row_sum = full ? tile_row_exp<true>(tS, valid, p.scale_log2, -m_run)
-                                 : tile_row_exp<false>(tS, valid, p.scale_log2, -m_run);
       tmem_st_wait();
-      l_run += row_sum;
+      l_run += part;
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
-    // epilogue: o = O / l, token-major f16
+    // epilogue: l = sum of the two halves; o = O / l for this half's 64 columns
     mbar_wait(&o_done[t], (T - 1) & 1, wg);
     tc_fence_after();
+    float* xb = xch + (T & 1) * 256;
+    xb[half * 128 + row] = l_run;
+    named_bar_sync(bar_id, 256);
+    const float l_row = l_run + xb[(half ^ 1) * 128 + row];
     const int qrow = qp * 256 + t * 128 + row;
-    const float inv_l = 1.0f / l_run;
-    __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128;
+    const float inv_l = 1.0f / l_row;
+    __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128 + col0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       uint32_t r[32];
-      tmem_ld32(tO + c * 32, r);
+      tmem_ld32(tO + col0 + c * 32, r);
       tmem_ld_wait();
       if (qrow < p.N) {
         uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
@@ -314,8 +344,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
       }
     }
-    if (p.lse && qrow < p.N)
-      p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    if (p.lse && half == 0 && qrow < p.N)
+      p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = (m_run + __log2f(l_row)) * 0.69314718055994531f;
   }
   tc_fence_before();
   __syncthreads();
