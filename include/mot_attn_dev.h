@@ -18,10 +18,10 @@ extern "C" {
 
 /* d = A B^T on the tensor cores (the persistent tcgen05 GEMM used by the
  * layer's projections): a device [m, k], b device [n, k], both bf16
- * (is_bf16 != 0) or both f16; d device f32 [m, n].
- * Requires k % 64 == 0, n % 256 == 0, m >= 1. */
+ * (is_bf16 != 0) or both f16; d device f32 [m, n]; output tiles 128 x tile_n
+ * (tile_n 128 or 256). Requires k % 64 == 0, n % tile_n == 0, m >= 1. */
 mot_status mot_dev_gemm(const void* a, const void* b, float* d, int32_t m, int32_t n, int32_t k,
-                        int32_t is_bf16, void* stream);
+                        int32_t is_bf16, int32_t tile_n, void* stream);
 
 /* Byte offsets, inside the `saved` buffer of a training forward, of the
  * activations it keeps (all device, f16 unless noted):

@@ -1088,15 +1088,16 @@ extern "C" mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int3
 extern "C" {
 
 mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, int32_t n, int32_t k, int32_t is_bf16,
-                        void* stream) {
+                        int32_t tile_n, void* stream) {
   if (!a || !b || !dmat || m <= 0 || n <= 0 || k <= 0) return MOT_ERR_INVALID_ARGUMENT;
-  if (k % 64 != 0 || n % 256 != 0) return MOT_ERR_UNSUPPORTED_SHAPE;
+  if (tile_n != 128 && tile_n != 256) return MOT_ERR_INVALID_ARGUMENT;
+  if (k % 64 != 0 || n % tile_n != 0) return MOT_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(a) || !aligned16(b) || !aligned16(dmat)) return MOT_ERR_ALIGNMENT;
   GemmCore core;
   const bool bf = is_bf16 != 0;
-  core_init(core, m, n, 256, 256, nullptr);
-  if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, 256)) return MOT_ERR_CUDA;
-  core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(128, 256, bf, bf), false, false);
+  core_init(core, m, n, tile_n, tile_n, nullptr);
+  if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, tile_n)) return MOT_ERR_CUDA;
+  core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(128, tile_n, bf, bf), false, false);
   core.num_segs = 1;
   EpiStore::Params ep = store_params(m, n);
   ep.out32 = dmat;
@@ -1104,9 +1105,9 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, in
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return launch_gemm<256, 4, EpiStore>(core, ep, sms, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MOT_OK
-             : MOT_ERR_CUDA;
+  const cudaError_t e = tile_n == 256 ? launch_gemm<256, 4, EpiStore>(core, ep, sms, static_cast<cudaStream_t>(stream))
+                                      : launch_gemm<128, 6, EpiStore>(core, ep, sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
 }
 
 mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream) {

@@ -107,10 +107,10 @@ def mot_status_string(status: int) -> str:
     return lib().mot_status_string(status).decode()
 
 
-def mot_dev_gemm(a, b, d, stream=None) -> None:
+def mot_dev_gemm(a, b, d, tile_n=256, stream=None) -> None:
     m, k = a.shape
     n = b.shape[0]
-    check(lib().mot_dev_gemm(_ptr(a), _ptr(b), _ptr(d), m, n, k, int(a.dtype == torch.bfloat16),
+    check(lib().mot_dev_gemm(_ptr(a), _ptr(b), _ptr(d), m, n, k, int(a.dtype == torch.bfloat16), tile_n,
                              _stream(stream)), "mot_dev_gemm")
 
 
