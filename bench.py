@@ -39,8 +39,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the 2048^2 CFG workload, keyed by the sha256 of the
 # kernel's source file at capture time: a changed kernel reports null.
 TRAFFIC = {
-    "attn_fwd": {"sha256": "6877987e024f348e6437d4696ef38d21d6ecef3ec714f3f9e9f46d781518cf00",
-                 "bytes": 104920576 + 34853632},
+    "attn_fwd": {"sha256": "455925fac2614ce6a7ded279b5b33f1c00db2d54c4046cd29f681133c7fc33b2",
+                 "bytes": 104929024 + 32312832},
+    "qkv_gemm": {"sha256": "a3e27cc7e03cf01608307002321cef734c2a77a5a52b7c90a6c75e27712b49b3",
+                 "bytes": 249139456 + 81316096},
 }
 KERNEL_SOURCES = {"attn_fwd": "attn_fwd.cuh", "qkv_gemm": "gemm.cuh", "o_gemm": "gemm.cuh"}
 
@@ -238,12 +240,27 @@ def run_once(args):
     layer = MotAttnLayer(wts, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_batch=wl.batch,
                          max_img_tokens=wl.img_tokens, max_prefix=wl.prefix)
     pl = [int(v) for v in td["prefix_len"]]
-    for _ in range(2):
-        y = layer.forward(td["x"], td["k_cache"], td["v_cache"], pl)
+    if args.train:
+        # forward keeping activations + backward, twice (the second is the one to capture)
+        layer.close()
+        layer = MotAttnLayer(wts, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_batch=wl.batch,
+                             max_img_tokens=wl.img_tokens, max_prefix=wl.prefix, enable_backward=True)
+        sv = layer.new_saved(wl.batch, wl.img_tokens, wl.prefix)
+        names = ("q", "k", "v", "o")
+        d_a = [torch.zeros(td["a_" + n].shape, device="cuda") for n in names] if wl.lora_rank else None
+        d_b = [torch.zeros(td["b_" + n].shape, device="cuda") for n in names] if wl.lora_rank else None
+        dy = td.get("dy", torch.randn_like(td["x"]))
+        for _ in range(2):
+            y = layer.forward(td["x"], td["k_cache"], td["v_cache"], pl, saved=sv)
+            dx = layer.backward(dy, td["x"], td["k_cache"], td["v_cache"], pl, sv, d_a=d_a, d_b=d_b)
+    else:
+        for _ in range(2):
+            y = layer.forward(td["x"], td["k_cache"], td["v_cache"], pl)
     torch.cuda.synchronize()
     status = layer.device_status()
     layer.close()
-    print(json.dumps({"once": wl.name, "status": status, "y_abs_mean": float(y.float().abs().mean())}))
+    print(json.dumps({"once": wl.name, "train": bool(args.train), "status": status,
+                      "y_abs_mean": float(y.float().abs().mean())}))
     return 0 if status == 0 else 1
 
 
@@ -525,6 +542,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--once", action="store_true", help="one warm forward, no timing (ncu target)")
     ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX)
+    ap.add_argument("--train", action="store_true", help="with --once: forward keeping activations + backward")
     args = ap.parse_args()
     if args.once:
         return run_once(args)
