@@ -15,6 +15,8 @@
 //   attn_bwd_dkv_kernel -- one CTA per (branch, KV head, 128-self-key tile),
 //                          loops over the group's query heads and query tiles:
 //                          S^T, dP^T, then dV += P^T dO and dK += dS^T q^.
+// The element-wise step needs no row reduction (lse and D were saved), so
+// each row is split over two threads of 64 columns each (8 warps).
 // dScore is multiplied by 2^10 (exact) before its f16 rounding so that small
 // probabilities stay normal in f16; the write-out multiplies by 2^-10.
 // The write-out applies RoPE^-1 (rotation by -angle) and the RMSNorm
@@ -47,6 +49,8 @@ struct AttnBwdParams {
   __half* dqkv;        // [B*N, (Hq+2Hkv)*dh] pre-norm gradients of q | k | v
   int* status;
 };
+
+constexpr int kAttnBwdThreads = 320;  // TMA warp, MMA warp, 8 element-wise warps
 
 struct AttnBwdSmem {
   static constexpr uint32_t kTile = 32768;
@@ -134,6 +138,15 @@ __device__ __forceinline__ void head_grad_writeout(uint32_t taddr, float scale, 
   }
 }
 
+// write 64 f16 values (32 packed words) as columns [64 half, 64 half + 64) of
+// row `row` of a 128x128 K-major 128-byte-swizzled tile (box `half`)
+__device__ __forceinline__ void store_swizzled_half_row(uint8_t* tile, int row, int half, const uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(tile + half * 16384 + row * 128 + ((c ^ (row & 7)) << 4)) =
+        make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+}
+
 // write 128 f16 values (64 packed words) as row `row` of a 128x128 K-major
 // 128-byte-swizzled tile (two 64-column boxes)
 __device__ __forceinline__ void store_swizzled_row(uint8_t* tile, int row, const uint32_t (&pk)[64]) {
@@ -149,7 +162,7 @@ __device__ __forceinline__ void store_swizzled_row(uint8_t* tile, int row, const
 }
 
 // ------------------------------------------------------------------ dq
-__global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdParams p) {
+__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr uint32_t T32 = AttnBwdSmem::kTile;
@@ -187,13 +200,13 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_consta
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&ds_full[i], 128);
+      mbar_init(&ds_full[i], 256);
       mbar_init(&ds_free[i], 1);
     }
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
     mbar_init(sdp_full, 1);
-    mbar_init(sdp_free, 128);
+    mbar_init(sdp_free, 256);
     mbar_init(dq_full, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -268,6 +281,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_consta
     }
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // key columns [64 half, 64 half + 64) of each tile
     const int row = quarter * 32 + lane;
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     const int n = qt * 128 + row;
@@ -281,9 +295,10 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_consta
       mbar_wait(sdp_full, j & 1, wg);
       tc_fence_after();
       const int valid_keys = L - j * 128;
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = half * 2 + cc;
         uint32_t rs[32], rd[32];
         tmem_ld32(tS + lo + c * 32, rs);
         tmem_ld32(tDP + lo + c * 32, rd);
@@ -298,19 +313,19 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_consta
           const float d0 = p0 * (__uint_as_float(rd[i]) - drow) * kDsScale;
           const float d1 = p1 * (__uint_as_float(rd[i + 1]) - drow) * kDsScale;
           overflow |= !(fabsf(d0) <= 65504.f) || !(fabsf(d1) <= 65504.f);
-          pk[c * 16 + i / 2] = pack_half2(d0, d1);
+          pk[cc * 16 + i / 2] = pack_half2(d0, d1);
         }
       }
       tc_fence_before();
       mbar_arrive(sdp_free);
       if (j >= 2) mbar_wait(&ds_free[s], ((j - 2) >> 1) & 1, wg);
-      store_swizzled_row(sDS + s * T32, row, pk);
+      store_swizzled_half_row(sDS + s * T32, row, half, pk);
       fence_proxy_async_smem();
       mbar_arrive(&ds_full[s]);
     }
     mbar_wait(dq_full, 0, wg);
     tc_fence_after();
-    {
+    if (half == 0) {
       const long long m = static_cast<long long>(b) * p.N + (valid ? n : 0);
       const int pos = p.plen[b] + (valid ? n : 0);
       const int hk = p.Hq + p.Hkv;
@@ -329,7 +344,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------------ dk, dv
-__global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdParams p) {
+__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr uint32_t T32 = AttnBwdSmem::kTile;
@@ -368,10 +383,10 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
       mbar_init(&qd_empty[i], 1);
     }
     mbar_init(sdp_full, 1);
-    mbar_init(sdp_free, 128);
-    mbar_init(pt_full, 128);
+    mbar_init(sdp_free, 256);
+    mbar_init(pt_full, 256);
     mbar_init(pt_free, 1);
-    mbar_init(dst_full, 128);
+    mbar_init(dst_full, 256);
     mbar_init(dst_free, 1);
     mbar_init(acc_full, 1);
     *abort_flag = 0u;
@@ -451,6 +466,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
     }
   } else {
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // query columns [64 half, 64 half + 64) of each tile
     const int row = quarter * 32 + lane;
     const uint32_t lo = static_cast<uint32_t>(quarter * 32) << 16;
     bool overflow = false;
@@ -458,12 +474,12 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
       const int h = g * G + it / p.q_tiles, qi = it % p.q_tiles;
       const long long sbase = (static_cast<long long>(b) * p.Hq + h) * p.N + qi * 128;
       const int qvalid = p.N - qi * 128;
-      // softmax statistics of this tile's 128 queries: lane l holds queries
-      // l, l+32, l+64, l+96; column c is read from lane c%32 by a shuffle
-      float lse_r[4], del_r[4];
+      // softmax statistics of this thread's 64 queries: lane l holds queries
+      // 64 half + l and 64 half + 32 + l; column c is read from lane c%32 by a shuffle
+      float lse_r[2], del_r[2];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int q = lane + 32 * k;
+      for (int k = 0; k < 2; ++k) {
+        const int q = half * 64 + lane + 32 * k;
         lse_r[k] = q < qvalid ? p.lse[sbase + q] * kLog2e : 0.f;
         del_r[k] = q < qvalid ? p.delta[sbase + q] : 0.f;
       }
@@ -471,22 +487,24 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
       tc_fence_after();
       // the A buffer holds dScore^T of the previous iteration until its dK MMA is done
       if (it >= 1) mbar_wait(dst_free, (it - 1) & 1, wg);
-      uint32_t dk[64];
+      uint32_t dk[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // 16-column chunks
+      for (int c = 0; c < 4; ++c) {  // 16-column chunks of this half
+        const int col0 = half * 64 + c * 16;
         uint32_t rs[16], rd[16];
-        tmem_ld16(tST + lo + c * 16, rs);
-        tmem_ld16(tDPT + lo + c * 16, rd);
+        tmem_ld16(tST + lo + col0, rs);
+        tmem_ld16(tDPT + lo + col0, rd);
         tmem_ld_wait();
         uint32_t pp[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const int col = c * 16 + i;
+          const int lc = c * 16 + i;  // column within this half
+          const int col = half * 64 + lc;
           const bool v0 = col < qvalid, v1 = col + 1 < qvalid;
-          const float l0 = __shfl_sync(0xffffffffu, lse_r[col >> 5], col & 31);
-          const float l1 = __shfl_sync(0xffffffffu, lse_r[(col + 1) >> 5], (col + 1) & 31);
-          const float D0 = __shfl_sync(0xffffffffu, del_r[col >> 5], col & 31);
-          const float D1 = __shfl_sync(0xffffffffu, del_r[(col + 1) >> 5], (col + 1) & 31);
+          const float l0 = __shfl_sync(0xffffffffu, lse_r[lc >> 5], lc & 31);
+          const float l1 = __shfl_sync(0xffffffffu, lse_r[(lc + 1) >> 5], (lc + 1) & 31);
+          const float D0 = __shfl_sync(0xffffffffu, del_r[lc >> 5], lc & 31);
+          const float D1 = __shfl_sync(0xffffffffu, del_r[(lc + 1) >> 5], (lc + 1) & 31);
           float p0 = ex2_approx(fmaf(__uint_as_float(rs[i]), p.scale_log2, -l0));
           float p1 = ex2_approx(fmaf(__uint_as_float(rs[i + 1]), p.scale_log2, -l1));
           p0 = v0 ? p0 : 0.f;
@@ -497,12 +515,11 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
           pp[i / 2] = pack_half2(p0, p1);
           dk[c * 8 + i / 2] = pack_half2(d0, d1);
         }
-        // P^T columns [16c, 16c+16) = two 16-byte chunks of the A buffer
+        // P^T columns [col0, col0+16) = two 16-byte chunks of box `half`
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
-          const int chunk = c * 2 + q2;
-          const int hf = chunk >> 3, cc = chunk & 7;
-          *reinterpret_cast<uint4*>(sA + hf * 16384 + row * 128 + ((cc ^ (row & 7)) << 4)) =
+          const int cc = c * 2 + q2;
+          *reinterpret_cast<uint4*>(sA + half * 16384 + row * 128 + ((cc ^ (row & 7)) << 4)) =
               make_uint4(pp[q2 * 4 + 0], pp[q2 * 4 + 1], pp[q2 * 4 + 2], pp[q2 * 4 + 3]);
         }
       }
@@ -511,7 +528,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
       fence_proxy_async_smem();
       mbar_arrive(pt_full);
       mbar_wait(pt_free, it & 1, wg);
-      store_swizzled_row(sA, row, dk);
+      store_swizzled_half_row(sA, row, half, dk);
       fence_proxy_async_smem();
       mbar_arrive(dst_full);
     }
@@ -522,19 +539,25 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkv_kernel(const __grid_const
     const long long m = static_cast<long long>(b) * p.N + (valid ? n : 0);
     const int hk = p.Hq + p.Hkv;
     const int ld = (p.Hq + 2 * p.Hkv) * 128;
-    head_grad_writeout(tDK + lo, p.inv_sqrt_dh / kDsScale, valid, p.rope + static_cast<long long>(pl + (valid ? n : 0)) * 64,
-                       p.gamma_k, p.xhat + (m * hk + p.Hq + g) * 128, valid ? p.rstd[m * hk + p.Hq + g] : 0.f,
-                       p.dqkv + m * ld + (p.Hq + g) * 128, overflow);
-    __half* dv = p.dqkv + m * ld + (p.Hq + p.Hkv + g) * 128;
+    if (half == 0) {
+      // dk: RoPE^-1 + RMSNorm backward
+      head_grad_writeout(tDK + lo, p.inv_sqrt_dh / kDsScale, valid,
+                         p.rope + static_cast<long long>(pl + (valid ? n : 0)) * 64, p.gamma_k,
+                         p.xhat + (m * hk + p.Hq + g) * 128, valid ? p.rstd[m * hk + p.Hq + g] : 0.f,
+                         p.dqkv + m * ld + (p.Hq + g) * 128, overflow);
+    } else {
+      // dv: stored as is
+      __half* dv = p.dqkv + m * ld + (p.Hq + p.Hkv + g) * 128;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t r16[16];
-      tmem_ld16(tDV + lo + c * 16, r16);
-      tmem_ld_wait();
-      float v[16];
+      for (int c = 0; c < 8; ++c) {
+        uint32_t r16[16];
+        tmem_ld16(tDV + lo + c * 16, r16);
+        tmem_ld_wait();
+        float v[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r16[i]);
-      if (valid) store_f16x16(dv + c * 16, v, overflow);
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r16[i]);
+        if (valid) store_f16x16(dv + c * 16, v, overflow);
+      }
     }
     if (overflow) atomicOr(p.status, DEV_ERR_NUMERIC);
   }

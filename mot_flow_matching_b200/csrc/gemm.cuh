@@ -269,6 +269,202 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   }
 }
 
+// ------------------------------------------------------------------ 2-SM variant
+// The same GEMM on CTA pairs (clusters of 2, tcgen05 cta_group::2): a pair
+// owns a 256 x BN output tile; CTA r of the pair stages rows [128r, 128r+128)
+// of A and rows [r BN/2, (r+1) BN/2) of B in its own shared memory, the even
+// CTA issues M=256 MMAs that read both CTAs' halves, and each CTA's TMEM
+// receives its 128 rows of D (all BN columns). Per SM this halves the B bytes
+// that TMA writes into, and the tensor core reads out of, shared memory.
+// Both CTAs' TMA loads complete on the even CTA's "full" barrier; MMA
+// completion is multicast to both CTAs' "empty" / "tfull" barriers; each
+// epilogue warp reports a drained accumulator to the even CTA's "tempty".
+template <int BN, int STAGES>
+struct Gemm2Smem {
+  static constexpr uint32_t kABytes = kBM * kBK * 2;        // this CTA's 128 rows of A
+  static constexpr uint32_t kBBytes = (BN / 2) * kBK * 2;   // this CTA's BN/2 rows of B
+  static constexpr uint32_t kBarOffset = STAGES * (kABytes + kBBytes);
+  static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;
+};
+
+template <int BN, int STAGES, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm2_kernel(const __grid_constant__ GemmArgs<Epi> args) {
+  static_assert(BN % 128 == 0 && BN <= 256, "two 64-column boxes of B per CTA half");
+  using L = Gemm2Smem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = tmem_cols_for(2 * BN);
+  constexpr int kHalfN = BN / 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const GemmCore& g = args.core;
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // the leader's expect_tx; both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one multicast commit per round
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // one arrive per epilogue warp of both CTAs
+    }
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int si = 0; si < g.num_segs; ++si) {
+      tma_prefetch_desc(&g.maps[g.segs[si].a_map]);
+      for (int r = 0; r < g.num_regions; ++r) tma_prefetch_desc(&g.maps[g.segs[si].b_map[r]]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barrier inits and the TMEM address visible to both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitGuard wg{abort_flag, g.status};
+
+  const int num_tiles = g.tiles_m * g.tiles_n;  // 256-row tiles
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+  const int num_segs = g.num_segs;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const int b_box_rows = g.b_box_rows;  // K-major B: rows per box (<= BN/2)
+      for (int tile = cluster; tile < num_tiles; tile += clusters) {
+        int tm, tn;
+        tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+        const int m0 = tm * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int n0 = tn * BN + static_cast<int>(rank) * kHalfN;
+        const int reg0 = region_of(g, tn * BN);
+        for (int si = 0; si < num_segs; ++si) {
+          const GemmSeg& sg = g.segs[si];
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb, a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
+          const CUtensorMap* amap = &g.maps[sg.a_map];
+          const int box_n = b_mn ? 64 : b_box_rows;
+          const int nbox = kHalfN / box_n;
+          const CUtensorMap* bmap[2];
+          int bcoord[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int n = n0 + (i < nbox ? i : 0) * box_n;
+            const int r = region_of(g, n);
+            bmap[i] = &g.maps[sg.b_map[r]];
+            bcoord[i] = n - g.region_n0[r];
+          }
+          const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
+          for (int kb = 0; kb < nkb; ++kb) {
+            mbar_wait(&empty[stage], phase ^ 1u, wg);
+            const uint32_t fbar = map_to_rank(smem_u32(&full[stage]), 0);
+            if (leader) mbar_expect_tx(&full[stage], 2 * (L::kABytes + L::kBBytes));
+            uint8_t* a_dst = sA + stage * L::kABytes;
+            uint8_t* b_dst = sB + stage * L::kBBytes;
+            const int ka = a_k0 + kb * kBK, kbk = b_k0 + kb * kBK;
+            if (a_mn) {
+              tma_load_2d_pair(a_dst, amap, fbar, m0, ka);
+              tma_load_2d_pair(a_dst + kMnBoxBytes, amap, fbar, m0 + 64, ka);
+            } else {
+              tma_load_2d_pair(a_dst, amap, fbar, ka, m0);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              if (i >= nbox) break;
+              if (b_mn)
+                tma_load_2d_pair(b_dst + i * box_bytes, bmap[i], fbar, bcoord[i], kbk);
+              else
+                tma_load_2d_pair(b_dst + i * box_bytes, bmap[i], fbar, kbk, bcoord[i]);
+            }
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = cluster; tile < num_tiles; tile += clusters) {
+        mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        uint32_t accumulate = 0u;
+        for (int si = 0; si < num_segs; ++si) {
+          const GemmSeg& sg = g.segs[si];
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb;
+          const uint32_t idesc = sg.idesc;  // built for M = 256, N = BN
+          for (int kb = 0; kb < nkb; ++kb) {
+            mbar_wait(&full[stage], phase, wg);
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
+            const uint32_t b_addr = smem_u32(sB + stage * L::kBBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = a_mn ? mnmajor_desc(a_addr, kk, kMnBoxBytes) : kmajor_desc(a_addr, kk, L::kABytes);
+              const uint64_t bd = b_mn ? mnmajor_desc(b_addr, kk, kMnBoxBytes) : kmajor_desc(b_addr, kk, L::kBBytes);
+              umma_ss_pair(d_tmem, ad, bd, idesc, accumulate);
+              accumulate = 1u;
+            }
+            umma_commit_pair(&empty[stage], 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < num_tiles; tile += clusters) {
+      int tm, tn;
+      tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+      mbar_wait(&tfull[acc], acc_phase, wg);
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
+      Epi::template apply<BN>(args.epi, taddr, tm * 2 * kBM + static_cast<int>(rank) * kBM, tn * BN, row, g.status);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // the peer's MMAs no longer read this CTA's shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ epilogues
 __device__ __forceinline__ void load_row32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];

@@ -191,6 +191,27 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   return cudaGetLastError();
 }
 
+// 2-SM (CTA pair) launch: core.tiles_m counts 256-row tiles
+template <int BN, int STAGES, class Epi>
+cudaError_t launch_gemm2(const GemmCore& core, const typename Epi::Params& ep, int num_sms, cudaStream_t st) {
+  static_assert(sizeof(GemmArgs<Epi>) <= 4096, "kernel parameter block");
+  using L = Gemm2Smem<BN, STAGES>;
+  static_assert(L::kBytes <= 232448, "shared memory");
+  auto kern = gemm2_kernel<BN, STAGES, Epi>;
+  static std::once_flag once;
+  std::call_once(once, [&] { set_smem_attr(kern, L::kBytes); });
+  GemmArgs<Epi> args;
+  args.core = core;
+  args.epi = ep;
+  const int tiles = core.tiles_m * core.tiles_n;
+  const int pairs = std::max(1, std::min(tiles, num_sms / 2));
+  kern<<<2 * pairs, kGemmThreads, L::kBytes, st>>>(args);
+  return cudaGetLastError();
+}
+
+// tiles of the pair kernel: 256 rows of D per CTA pair
+void core_pair(GemmCore& c) { c.tiles_m = (c.M + 2 * kBM - 1) / (2 * kBM); }
+
 // BN = 64 or 128 instantiation for the narrow (LoRA-rank-wide) GEMMs
 template <class Epi>
 cudaError_t launch_gemm_narrow(int BN, const GemmCore& core, const typename Epi::Params& ep, int num_sms,
@@ -249,11 +270,11 @@ void set_out16(EpiStore::Params& p, int i, void* ptr, long long ld, bool bf16, f
   p.o16[i].residual_of = residual_of;
 }
 
-// K-major f16 maps over the per-call f16 copies of lora_up (box rows 256)
+// K-major f16 maps over the per-call f16 copies of lora_up (box rows 128)
 bool lora_up16_maps(CUtensorMap* m, const __half* b16, int r, const int (&rows)[3]) {
   long long off = 0;
   for (int j = 0; j < 3; ++j) {
-    if (!map2d(&m[j], b16 + off, false, r, rows[j], r, 256)) return false;
+    if (!map2d(&m[j], b16 + off, false, r, rows[j], r, 128)) return false;
     off += static_cast<long long>(rows[j]) * r;
   }
   return true;
@@ -294,7 +315,7 @@ struct mot_attn {
   int stage_ids[kMaxStages] = {};
   int stage_count = 0;
   // forward weight maps (K-major)
-  CUtensorMap wq, wk, wv, wo;  // box rows 256
+  CUtensorMap wq, wk, wv, wo;  // box rows 128
   CUtensorMap aq, ak, av;      // lora_down q/k/v, box rows RP
   // backward weight maps (MN-major, 64 x 64 boxes)
   CUtensorMap wo_mn, ao_mn, bo_mn, wq16_mn, wk16_mn, wv16_mn, aq_mn, ak_mn, av_mn;
@@ -305,8 +326,8 @@ namespace {
 mot_status build_weight_maps(mot_attn* h) {
   const mot_attn_config& c = h->cfg;
   const uint64_t d = c.hidden, qd = c.n_q_heads * 128, kvd = c.n_kv_heads * 128;
-  bool ok = map2d(&h->wq, h->w.w_q, true, d, qd, d, 256) && map2d(&h->wk, h->w.w_k, true, d, kvd, d, 256) &&
-            map2d(&h->wv, h->w.w_v, true, d, kvd, d, 256) && map2d(&h->wo, h->wo16, false, qd, d, qd, 256);
+  bool ok = map2d(&h->wq, h->w.w_q, true, d, qd, d, 128) && map2d(&h->wk, h->w.w_k, true, d, kvd, d, 128) &&
+            map2d(&h->wv, h->w.w_v, true, d, kvd, d, 128) && map2d(&h->wo, h->wo16, false, qd, d, qd, 128);
   if (ok && h->rank > 0) {
     const uint64_t r = h->rank;
     const uint32_t box_a = static_cast<uint32_t>(h->RP);
@@ -600,7 +621,8 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   lz.stage = ST_QKV_GEMM;
   {
     GemmCore core;
-    core_init(core, M, nqkv, 256, 256, h->status);
+    core_init(core, M, nqkv, 256, 128, h->status);
+    core_pair(core);
     bool ok = map2d(&core.maps[0], x, true, d, M, d, 128);
     if (r > 0)
       ok = ok && map2d(&core.maps[1], u_qkv, false, 3 * RP, M, 3 * RP, 128) &&
@@ -614,11 +636,11 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     core.region_n0[1] = qd;
     core.region_n0[2] = qd + kvd;
     core.region_n0[3] = nqkv;
-    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, 256, true, true), false, false);
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(256, 256, true, true), false, false);
     for (int j = 0; j < 3; ++j) core.segs[0].b_map[j] = 2 + j;
     core.num_segs = 1;
     if (r > 0) {
-      core.segs[1] = seg1(1, 0, 5, RP / 64, idesc_f16(128, 256, false, false), false, false);
+      core.segs[1] = seg1(1, 0, 5, RP / 64, idesc_f16(256, 256, false, false), false, false);
       for (int j = 0; j < 3; ++j) {
         core.segs[1].a_k0[j] = j * RP;
         core.segs[1].b_map[j] = 5 + j;
@@ -641,7 +663,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ep.Lcap = L.Lcap;
     ep.M = M;
     ep.eps = c.rms_eps;
-    lz.done(launch_gemm<256, 4, EpiQkv>(core, ep, h->num_sms, st));
+    lz.done(launch_gemm2<256, 6, EpiQkv>(core, ep, h->num_sms, st));
   }
   // 5. attention
   lz.stage = ST_ATTN_FWD;
@@ -689,23 +711,24 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   lz.stage = ST_O_GEMM;
   {
     GemmCore core;
-    core_init(core, M, d, 256, 256, h->status);
+    core_init(core, M, d, 256, 128, h->status);
+    core_pair(core);
     bool ok = map2d(&core.maps[0], attn, false, qd, M, qd, 128);
     if (r > 0)
-      ok = ok && map2d(&core.maps[1], u_o, false, RP, M, RP, 128) && map2d(&core.maps[3], bo16, false, r, d, r, 256);
+      ok = ok && map2d(&core.maps[1], u_o, false, RP, M, RP, 128) && map2d(&core.maps[3], bo16, false, r, d, r, 128);
     if (!ok) return MOT_ERR_CUDA;
     core.maps[2] = h->wo;
-    core.segs[0] = seg1(0, 0, 2, qd / 64, idesc_f16(128, 256, false, false), false, false);
+    core.segs[0] = seg1(0, 0, 2, qd / 64, idesc_f16(256, 256, false, false), false, false);
     core.num_segs = 1;
     if (r > 0) {
-      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(128, 256, false, false), false, false);
+      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(256, 256, false, false), false, false);
       core.num_segs = 2;
     }
     EpiStore::Params ep = store_params(M, d);
     set_out16(ep, 0, y, d, true);
     ep.out32 = y_f32;
     ep.ld32 = d;
-    lz.done(launch_gemm<256, 4, EpiStore>(core, ep, h->num_sms, st));
+    lz.done(launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   return lz.finish();
 }
@@ -884,10 +907,10 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       set_smem_attr(attn_bwd_dkv_kernel, AttnBwdSmem::kBytes);
     });
     lz.stage = ST_BWD_DQ;
-    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, 192, AttnBwdSmem::kBytes, st>>>(ap);
+    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
     lz.stage = ST_BWD_DKV;
-    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, 192, AttnBwdSmem::kBytes, st>>>(ap);
+    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
   }
   if (r > 0) {
