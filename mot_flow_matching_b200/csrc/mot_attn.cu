@@ -822,22 +822,23 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
   lz.stage = ST_BWD_DO;
   {
     GemmCore core;
-    core_init(core, M, qd, 256, 256, h->status);
+    core_init(core, M, qd, 256, 128, h->status);
+    core_pair(core);
     bool ok = map2d(&core.maps[0], dy, true, d, M, d, 128);
     if (r > 0)
       ok = ok && map2d(&core.maps[1], g_ohi, true, RP, M, RP, 128) && map2d(&core.maps[4], g_olo, true, RP, M, RP, 128);
     if (!ok) return MOT_ERR_CUDA;
     core.maps[2] = h->wo_mn;
-    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(256, 256, true, true, false, true), false, true);
     core.num_segs = 1;
     if (r > 0) {
       core.maps[3] = h->ao_mn;
-      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
-      core.segs[2] = seg1(4, 0, 3, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+      core.segs[1] = seg1(1, 0, 3, RP / 64, idesc_f16(256, 256, true, true, false, true), false, true);
+      core.segs[2] = seg1(4, 0, 3, RP / 64, idesc_f16(256, 256, true, true, false, true), false, true);
       core.num_segs = 3;
     }
     EpiDattn::Params ep{dO, attn, delta, M, N, Hq};
-    lz.done(launch_gemm<256, 4, EpiDattn>(core, ep, h->num_sms, st));
+    lz.done(launch_gemm2<256, 6, EpiDattn>(core, ep, h->num_sms, st));
   }
   if (r > 0) {
     // dB_o = dy^T u_o   [d, r], with u_o as its bf16 hi + lo pair
@@ -981,7 +982,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
   lz.stage = ST_BWD_DX;
   {
     GemmCore core;
-    core_init(core, M, d, 256, 256, h->status);
+    core_init(core, M, d, 256, 128, h->status);
+    core_pair(core);
     bool ok = map2d(&core.maps[0], dqkv, false, nqkv, M, nqkv, 128);
     if (r > 0)
       ok = ok && map2d(&core.maps[1], g_hi, true, 3 * RP, M, 3 * RP, 128) &&
@@ -991,15 +993,15 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     core.maps[3] = h->wk16_mn;
     core.maps[4] = h->wv16_mn;
     for (int j = 0; j < 3; ++j)
-      core.segs[j] = seg1(0, col0[j], 2 + j, outj[j] / 64, idesc_f16(128, 256, false, false, false, true), false, true);
+      core.segs[j] = seg1(0, col0[j], 2 + j, outj[j] / 64, idesc_f16(256, 256, false, false, false, true), false, true);
     core.num_segs = 3;
     if (r > 0) {
       core.maps[5] = h->aq_mn;
       core.maps[6] = h->ak_mn;
       core.maps[7] = h->av_mn;
       for (int j = 0; j < 3; ++j) {
-        core.segs[3 + j] = seg1(1, j * RP, 5 + j, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
-        core.segs[6 + j] = seg1(8, j * RP, 5 + j, RP / 64, idesc_f16(128, 256, true, true, false, true), false, true);
+        core.segs[3 + j] = seg1(1, j * RP, 5 + j, RP / 64, idesc_f16(256, 256, true, true, false, true), false, true);
+        core.segs[6 + j] = seg1(8, j * RP, 5 + j, RP / 64, idesc_f16(256, 256, true, true, false, true), false, true);
       }
       core.num_segs = 9;
     }
@@ -1007,7 +1009,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     set_out16(ep, 0, dx, d, true);
     ep.out32 = dx_f32;
     ep.ld32 = d;
-    lz.done(launch_gemm<256, 4, EpiStore>(core, ep, h->num_sms, st));
+    lz.done(launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   return lz.finish();
 }
