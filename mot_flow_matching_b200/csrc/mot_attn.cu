@@ -901,17 +901,19 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     ap.gamma_k = h->gamma + 128;
     ap.rope = h->rope;
     ap.dqkv = dqkv;
+    ap.qhat = q_hat;
+    ap.dout = dO;
     ap.status = h->status;
     static std::once_flag once;
     std::call_once(once, [] {
-      set_smem_attr(attn_bwd_dq_kernel, AttnBwdSmem::kBytes);
-      set_smem_attr(attn_bwd_dkv_kernel, AttnBwdSmem::kBytes);
+      set_smem_attr(attn_bwd_dq_kernel, AttnBwdDqSmem::kBytes);
+      set_smem_attr(attn_bwd_dkv_kernel, AttnBwdDkvSmem::kBytes);
     });
     lz.stage = ST_BWD_DQ;
-    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
+    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdDqSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
     lz.stage = ST_BWD_DKV;
-    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
+    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, kAttnBwdThreads, AttnBwdDkvSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
   }
   if (r > 0) {
