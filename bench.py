@@ -96,10 +96,11 @@ def stage_work(wl, stage):
         return 2.0 * M * hid * r, 2.0 * (M * hid + M * r)
     if stage == "bwd_da_o":
         return 2.0 * M * Hq * dh * r, 2.0 * (M * Hq * dh + M * r)
-    if stage == "attn_bwd_dq":   # S, dP and dQ over all L keys
-        return 6.0 * B * Hq * N * L * dh, 2.0 * (2 * B * Hq * N * dh + 2 * B * Hkv * L * dh + M * qkv)
-    if stage == "attn_bwd_dkv":  # dK and dV over the N self keys (S, dP recomputed on top)
-        return 4.0 * B * Hq * N * N * dh, 2.0 * (2 * B * Hq * N * dh + 2 * B * Hkv * N * dh)
+    if stage == "attn_bwd":
+        # S, dP and dQ over all L keys; dK and dV over the N self keys (the
+        # dk/dv CTAs recompute S^T and dP^T on top: not counted)
+        return (6.0 * B * Hq * N * L * dh + 4.0 * B * Hq * N * N * dh,
+                2.0 * (2 * B * Hq * N * dh + 2 * B * Hkv * L * dh + M * qkv))
     if stage in ("bwd_g_qkv", "bwd_db_qkv"):
         return 2.0 * M * qkv * r / 3.0, 2.0 * (M * qkv + M * r) / 3.0
     if stage == "bwd_da_qkv":

@@ -8,13 +8,13 @@
 // the N self keys (the cache is constant). With P = softmax(q^K^T/sqrt(dh)),
 // D = rowsum(dO * O) and dScore = P * (dO V^T - D):
 //   dq^ = dScore K / sqrt(dh),  dk^ = dScore^T q^ / sqrt(dh),  dv = P^T dO.
-// Two kernels keep every sum in a fixed order (no atomics, bitwise
-// deterministic):
-//   attn_bwd_dq_kernel  -- one CTA per (branch, query head, 128-query tile).
+// Two kinds of CTA, in one launch, keep every sum in a fixed order (no
+// atomics, bitwise deterministic):
+//   dq CTAs  -- one CTA per (branch, query head, 128-query tile).
 //       q^ and dO of the tile sit in TMEM as the A operands of S = q^ K^T and
 //       dP = dO V^T, so only K and V stream through shared memory. dScore is
 //       written over the dP columns and feeds dQ += dScore K from TMEM.
-//   attn_bwd_dkv_kernel -- one CTA per (branch, KV head, 128-self-key tile),
+//   dk/dv CTAs -- one CTA per (branch, KV head, 128-self-key tile),
 //       looping over the group's query heads and query tiles: S^T, dP^T, then
 //       P^T written over S^T feeds dV += P^T dO and dScore^T written over dP^T
 //       feeds dK += dScore^T q^, both with the A operand in TMEM.
@@ -48,6 +48,7 @@ struct AttnBwdParams {
   const __half* qhat;  // [B*Hq, N, dh]
   const __half* dout;  // [B*N, Hq*dh]
   int B, N, Hq, Hkv, Lcap, q_tiles, kv_tiles;
+  int dkv_ctas;  // B * Hkv * kv_tiles
   int plen[kMaxBatch];
   float scale_log2;  // log2(e) / sqrt(dh)
   float inv_sqrt_dh;
@@ -179,9 +180,7 @@ __device__ __forceinline__ void exp2_pair(float& p0, float& p1, float x0, float 
 }
 
 // ------------------------------------------------------------------ dq
-__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ void attn_bwd_dq_cta(const AttnBwdParams& p, int bid, uint8_t* smem) {
   constexpr uint32_t T32 = AttnBwdDqSmem::kTile;
   uint8_t* sK = smem + AttnBwdDqSmem::kK;
   uint8_t* sV = smem + AttnBwdDqSmem::kV;
@@ -200,7 +199,6 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dq_kernel(const _
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = warp_id(), lane = lane_id();
-  int bid = blockIdx.x;
   const int qt = bid % p.q_tiles;
   bid /= p.q_tiles;
   const int h = bid % p.Hq;
@@ -419,9 +417,7 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dq_kernel(const _
 }
 
 // ------------------------------------------------------------------ dk, dv
-__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ void attn_bwd_dkv_cta(const AttnBwdParams& p, int bid, uint8_t* smem) {
   constexpr uint32_t T32 = AttnBwdDkvSmem::kTile;
   uint8_t* sK = smem + AttnBwdDkvSmem::kK;
   uint8_t* sV = smem + AttnBwdDkvSmem::kV;
@@ -439,7 +435,6 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dkv_kernel(const 
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = warp_id(), lane = lane_id();
-  int bid = blockIdx.x;
   const int kt = bid % p.kv_tiles;
   bid /= p.kv_tiles;
   const int g = bid % p.Hkv;
@@ -669,6 +664,24 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_dkv_kernel(const 
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// One launch for both: blocks [0, dkv_ctas) take (branch, KV head, key
+// tile), the rest (branch, query head, query tile); the long dk/dv CTAs are
+// dispatched first and the short dq CTAs fill the SMs as they free up.
+struct AttnBwdSmem {
+  static constexpr uint32_t kBytes =
+      AttnBwdDqSmem::kBytes > AttnBwdDkvSmem::kBytes ? AttnBwdDqSmem::kBytes : AttnBwdDkvSmem::kBytes;
+};
+
+__global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int bid = static_cast<int>(blockIdx.x);
+  if (bid < p.dkv_ctas)
+    attn_bwd_dkv_cta(p, bid, smem);
+  else
+    attn_bwd_dq_cta(p, bid - p.dkv_ctas, smem);
 }
 
 }  // namespace mot

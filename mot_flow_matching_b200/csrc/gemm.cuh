@@ -55,6 +55,15 @@ struct GemmCore {
   int tiles_m, tiles_n;
   int b_box_rows;  // rows per K-major B TMA box; BN is a multiple of it
   int* status;
+  // split-K (1-CTA kernel only): work item = (tile, split); split s takes
+  // k-blocks [s total_kb / k_splits, (s+1) total_kb / k_splits) of the
+  // concatenated segments and writes its f32 partial tile to split_ws; the
+  // CTA that finishes a tile last (per-tile counter in split_cnt, which it
+  // resets) sums the partials in split order into TMEM and runs the epilogue.
+  int k_splits;  // 1 = off
+  int total_kb;
+  float4* split_ws;  // [tiles * k_splits][BN / 4][128]
+  int* split_cnt;    // [tiles], zero between launches
 };
 
 template <class Epi>
@@ -144,6 +153,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const WaitGuard wg{abort_flag, g.status};
 
   const int num_tiles = g.tiles_m * g.tiles_n;
+  const int splits = g.k_splits > 1 ? g.k_splits : 1;
+  const int num_items = num_tiles * splits;
+  const int total_kb = g.total_kb;
 
   // Both issuing threads copy what they need out of the parameter block into
   // registers before their K loops: the TMA / MMA wrappers clobber memory, so
@@ -154,14 +166,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       int stage = 0;
       uint32_t phase = 0;
       const int b_box_rows = g.b_box_rows;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+        const int tile = item / splits, split = item - tile * splits;
+        const int kb_lo = split * total_kb / splits, kb_hi = (split + 1) * total_kb / splits;
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
         const int m0 = tm * kBM, n0 = tn * BN;
         const int reg0 = region_of(g, n0);
+        int gk = 0;  // k-blocks of the segments before this one
         for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
           const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb, a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
+          const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);
+          gk += nkb;
           const CUtensorMap* amap = &g.maps[sg.a_map];
           // B boxes of this tile: up to 4 (map, row/column offset) pairs
           const int box_n = b_mn ? 64 : b_box_rows;
@@ -176,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             bcoord[i] = n - g.region_n0[r];
           }
           const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
-          for (int kb = 0; kb < nkb; ++kb) {
+          for (int kb = kb0; kb < kb1; ++kb) {
             mbar_wait(&empty[stage], phase ^ 1u, wg);
             mbar_expect_tx(&full[stage], L::kABytes + L::kBBytes);
             uint8_t* a_dst = sA + stage * L::kABytes;
@@ -210,16 +227,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+        const int split = item % splits;
+        const int kb_lo = split * total_kb / splits, kb_hi = (split + 1) * total_kb / splits;
         mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         uint32_t accumulate = 0u;
+        int gk = 0;
         for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
           const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb;
           const uint32_t idesc = sg.idesc;
-          for (int kb = 0; kb < nkb; ++kb) {
+          const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);
+          gk += nkb;
+          for (int kb = kb0; kb < kb1; ++kb) {
             mbar_wait(&full[stage], phase, wg);
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
@@ -248,13 +270,65 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+      const int tile = item / splits;
       int tm, tn;
       tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
       mbar_wait(&tfull[acc], acc_phase, wg);
       tc_fence_after();
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
-      Epi::template apply<BN>(args.epi, taddr, tm * kBM, tn * BN, row, g.status);
+      bool run_epi = true;
+      if (splits > 1) {
+        // this split's partial tile out, chunk-major so that a warp's stores are contiguous
+        float4* part = g.split_ws + static_cast<long long>(item) * (BN / 4) * kBM + row;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            __stcg(part + ((c >> 2) + i) * kBM, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                            __uint_as_float(r[4 * i + 2]),
+                                                            __uint_as_float(r[4 * i + 3])));
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) *last_flag = atomicAdd(g.split_cnt + tile, 1) == splits - 1;
+        named_bar_sync(1, 128);
+        run_epi = *last_flag != 0;
+        if (run_epi) {
+          // the tile's sum over splits, in split order, back into TMEM
+          __threadfence();
+          const float4* base = g.split_ws + static_cast<long long>(tile) * splits * (BN / 4) * kBM + row;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll 1
+            for (int sp = 0; sp < splits; ++sp) {
+              const float4* q = base + static_cast<long long>(sp) * (BN / 4) * kBM + (c >> 2) * kBM;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 f = __ldcg(q + i * kBM);
+                v[4 * i] += f.x;
+                v[4 * i + 1] += f.y;
+                v[4 * i + 2] += f.z;
+                v[4 * i + 3] += f.w;
+              }
+            }
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+            tmem_st32(taddr + c, w);
+          }
+          tmem_st_wait();
+          if (warp == 2 && lane == 0) g.split_cnt[tile] = 0;
+        }
+      }
+      if (run_epi) Epi::template apply<BN>(args.epi, taddr, tm * kBM, tn * BN, row, g.status);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;

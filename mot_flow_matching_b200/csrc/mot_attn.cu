@@ -93,6 +93,10 @@ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ------------------------------------------------------------------ layouts
+// split-K partial tiles of the LoRA-gradient GEMMs (backward workspace)
+constexpr size_t kSplitWsBytes = size_t(16) << 20;
+constexpr int kSplitCounters = 1024;
+
 struct Layout {
   int B = 0, N = 0, P = 0, M = 0, Lcap = 0, r = 0, RP = 0;
   // activations: in `saved` for training, else after the forward scratch
@@ -102,7 +106,7 @@ struct Layout {
   size_t w_ao16 = 0, w_bo16 = 0, w_bqkv16 = 0, fwd_scratch = 0;
   // backward scratch (workspace)
   size_t b_do = 0, b_delta = 0, b_dqkv = 0, b_gohi = 0, b_golo = 0, b_go16 = 0, b_ghi = 0, b_glo = 0, b_bqkv16 = 0,
-         bwd_scratch = 0;
+         b_split = 0, bwd_scratch = 0;
   size_t workspace() const { return std::max(fwd_scratch + act_bytes, bwd_scratch); }
 };
 
@@ -150,6 +154,7 @@ Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
   L.b_ghi = take(r ? M * 3 * RP * 2 : 0);
   L.b_glo = take(r ? M * 3 * RP * 2 : 0);
   L.b_bqkv16 = take(r ? nqkv * r * 2 : 0);
+  L.b_split = take(r ? kSplitWsBytes : 0);
   L.bwd_scratch = c.enable_backward ? off : 0;
   return L;
 }
@@ -174,6 +179,31 @@ void set_smem_attr(K kernel, size_t bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
+// Split count for a GEMM of `tiles` output tiles and total_kb k-blocks: the
+// fewest splits that come close to the best SM balance ceil(items/SMs)/S,
+// each split costing a little for its partial-tile round trip; at most 16,
+// at least two k-blocks per split, partials within the split workspace.
+int pick_splits(int tiles, int total_kb, int num_sms, int bn) {
+  int best = 1;
+  double best_cost = static_cast<double>((tiles + num_sms - 1) / num_sms);
+  for (int sp = 2; sp <= 16 && 2 * sp <= total_kb; ++sp) {
+    if (static_cast<size_t>(tiles) * sp * bn * kBM * 4 > kSplitWsBytes) break;
+    const double cost = static_cast<double>((tiles * sp + num_sms - 1) / num_sms) / sp + 0.02 * (sp - 1);
+    if (cost < best_cost - 1e-9) {
+      best = sp;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+// let launch_gemm split K (1-CTA kernel; partials in ws, counters in cnt)
+void enable_split(GemmCore& c, void* ws, int* cnt) {
+  c.k_splits = -1;
+  c.split_ws = static_cast<float4*>(ws);
+  c.split_cnt = cnt;
+}
+
 template <int BN, int STAGES, class Epi>
 cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, int num_sms, cudaStream_t st) {
   static_assert(sizeof(GemmArgs<Epi>) <= 4096, "kernel parameter block");
@@ -186,7 +216,13 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   args.core = core;
   args.epi = ep;
   const int tiles = core.tiles_m * core.tiles_n;
-  const int grid = std::max(1, std::min(tiles, num_sms));
+  int total_kb = 0;
+  for (int i = 0; i < core.num_segs; ++i) total_kb += core.segs[i].kb;
+  args.core.total_kb = total_kb;
+  args.core.k_splits =
+      core.k_splits < 0 && tiles <= kSplitCounters ? pick_splits(tiles, total_kb, num_sms, BN) : 1;
+  const int items = tiles * args.core.k_splits;
+  const int grid = std::max(1, std::min(items, num_sms));
   kern<<<grid, kGemmThreads, L::kBytes, st>>>(args);
   return cudaGetLastError();
 }
@@ -287,12 +323,11 @@ constexpr int kMaxStages = 32;
 enum StageId : int {
   ST_CVT_LORA_O = 0, ST_BUILD_KV = 1, ST_LORA_DOWN_QKV = 2, ST_QKV_GEMM = 3, ST_ATTN_FWD = 4,
   ST_LORA_DOWN_O = 5, ST_O_GEMM = 6, ST_BWD_CVT = 7, ST_BWD_G_O = 8, ST_BWD_DO = 9, ST_BWD_DB_O = 10,
-  ST_BWD_DA_O = 11, ST_BWD_DQ = 12, ST_BWD_DKV = 13, ST_BWD_G_QKV = 14, ST_BWD_DB_QKV = 15, ST_BWD_DA_QKV = 16,
-  ST_BWD_DX = 17,
+  ST_BWD_DA_O = 11, ST_BWD_ATTN = 12, ST_BWD_G_QKV = 13, ST_BWD_DB_QKV = 14, ST_BWD_DA_QKV = 15, ST_BWD_DX = 16,
 };
 const char* const kStageNames[] = {"cvt_lora_o", "build_kv", "lora_down_qkv", "qkv_gemm", "attn_fwd",
                                    "lora_down_o", "o_gemm", "bwd_cvt_lora", "bwd_g_o", "bwd_do_gemm",
-                                   "bwd_db_o", "bwd_da_o", "attn_bwd_dq", "attn_bwd_dkv", "bwd_g_qkv",
+                                   "bwd_db_o", "bwd_da_o", "attn_bwd", "bwd_g_qkv",
                                    "bwd_db_qkv", "bwd_da_qkv", "bwd_dx_gemm"};
 
 struct mot_attn {
@@ -307,6 +342,7 @@ struct mot_attn {
   float2* rope = nullptr;
   int rope_len = 0;
   int* status = nullptr;
+  int* split_cnt = nullptr;  // [kSplitCounters] per-tile split-K arrival counters (backward), zero at rest
   int num_sms = 148;
   int last_launches = 0;
   // optional per-launch timing (mot_dev_profile)
@@ -382,6 +418,7 @@ void release(mot_attn* h) {
   cudaFree(h->gamma);
   cudaFree(h->rope);
   cudaFree(h->status);
+  cudaFree(h->split_cnt);
   delete h;
 }
 
@@ -477,7 +514,10 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
   bool ok = cudaMalloc(&h->wo16, d * qd * 2) == cudaSuccess && cudaMalloc(&h->gamma, 2 * dh * 4) == cudaSuccess &&
             cudaMalloc(&h->rope, static_cast<size_t>(h->rope_len) * 64 * sizeof(float2)) == cudaSuccess &&
             cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
-  if (ok && cfg->enable_backward) ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess;
+  if (ok && cfg->enable_backward)
+    ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess &&
+         cudaMalloc(&h->split_cnt, kSplitCounters * sizeof(int)) == cudaSuccess &&
+         cudaMemset(h->split_cnt, 0, kSplitCounters * sizeof(int)) == cudaSuccess;
   if (!ok) {
     release(h);
     return MOT_ERR_CUDA;
@@ -783,6 +823,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
   __nv_bfloat16* g_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.b_ghi);
   __nv_bfloat16* g_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.b_glo);
   __half* b16 = reinterpret_cast<__half*>(ws + L.b_bqkv16);  // B_q|B_k|B_v in f16
+  void* split_ws = ws + L.b_split;
 
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M, RP = h->RP;
   const int qd = Hq * 128, kvd = Hkv * 128, nqkv = qd + 2 * kvd;
@@ -816,6 +857,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     set_out16(ep, 1, g_olo, RP, true, 1.0f, 0);
     set_out16(ep, 2, g_o16, RP, false, h->scale);
     ep.check_f16 = 1;
+    enable_split(core, split_ws, h->split_cnt);
     lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
   }
   // dO = dy W_o + s g_o A_o (f16) and D = rowsum(dO o)
@@ -856,6 +898,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.out32 = d_b[3];
       ep.ld32 = r;
       ep.accumulate32 = accumulate;
+      enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
     // dA_o = (s g_o)^T o   [r, qd], computed as its transpose o^T (s g_o)
@@ -872,6 +915,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.ld32 = qd;
       ep.accumulate32 = accumulate;
       ep.transpose32 = 1;
+      enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
   }
@@ -890,6 +934,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     ap.Lcap = L.Lcap;
     ap.q_tiles = (N + 127) / 128;
     ap.kv_tiles = (N + 127) / 128;
+    ap.dkv_ctas = B * Hkv * ap.kv_tiles;
     for (int b = 0; b < B; ++b) ap.plen[b] = prefix_len[b];
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
     ap.inv_sqrt_dh = static_cast<float>(1.0 / std::sqrt(128.0));
@@ -905,15 +950,9 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     ap.dout = dO;
     ap.status = h->status;
     static std::once_flag once;
-    std::call_once(once, [] {
-      set_smem_attr(attn_bwd_dq_kernel, AttnBwdDqSmem::kBytes);
-      set_smem_attr(attn_bwd_dkv_kernel, AttnBwdDkvSmem::kBytes);
-    });
-    lz.stage = ST_BWD_DQ;
-    attn_bwd_dq_kernel<<<B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdDqSmem::kBytes, st>>>(ap);
-    lz.done(cudaGetLastError());
-    lz.stage = ST_BWD_DKV;
-    attn_bwd_dkv_kernel<<<B * Hkv * ap.kv_tiles, kAttnBwdThreads, AttnBwdDkvSmem::kBytes, st>>>(ap);
+    std::call_once(once, [] { set_smem_attr(attn_bwd_kernel, AttnBwdSmem::kBytes); });
+    lz.stage = ST_BWD_ATTN;
+    attn_bwd_kernel<<<ap.dkv_ctas + B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
     lz.done(cudaGetLastError());
   }
   if (r > 0) {
@@ -939,6 +978,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       EpiStore::Params ep = store_params(M, 3 * RP);
       set_out16(ep, 0, g_hi, 3 * RP, true, h->scale);
       set_out16(ep, 1, g_lo, 3 * RP, true, 1.0f, 0);
+      enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
     for (int j = 0; j < 3; ++j) {
@@ -955,6 +995,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.out32 = d_b[j];
       ep.ld32 = r;
       ep.accumulate32 = accumulate;
+      enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
     {
@@ -977,6 +1018,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.M = d;
       ep.transpose = 1;
       ep.accumulate = accumulate;
+      enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiLoraGrad>(RP, core, ep, h->num_sms, st));
     }
   }
