@@ -154,7 +154,7 @@ Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
   L.b_ghi = take(r ? M * 3 * RP * 2 : 0);
   L.b_glo = take(r ? M * 3 * RP * 2 : 0);
   L.b_bqkv16 = take(r ? nqkv * r * 2 : 0);
-  L.b_split = take(r ? kSplitWsBytes : 0);
+  L.b_split = take(r ? 2 * kSplitWsBytes : 0);  // caller's stream, side stream
   L.bwd_scratch = c.enable_backward ? off : 0;
   return L;
 }
@@ -342,12 +342,17 @@ struct mot_attn {
   float2* rope = nullptr;
   int rope_len = 0;
   int* status = nullptr;
-  int* split_cnt = nullptr;  // [kSplitCounters] per-tile split-K arrival counters (backward), zero at rest
+  int* split_cnt = nullptr;  // [2][kSplitCounters] split-K arrival counters (backward; caller's / side stream)
   int num_sms = 148;
   int last_launches = 0;
-  // optional per-launch timing (mot_dev_profile)
+  // backward: a second stream for the gradient GEMMs nothing later depends on
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  // optional per-launch timing (mot_dev_profile): a start and an end event
+  // per launch, on the stream it ran on
   bool profile = false;
-  cudaEvent_t ev[kMaxStages + 1] = {};
+  cudaEvent_t ev[2 * kMaxStages + 2] = {};
+  cudaEvent_t stage_start[kMaxStages] = {}, stage_end[kMaxStages] = {};
   int stage_ids[kMaxStages] = {};
   int stage_count = 0;
   // forward weight maps (K-major)
@@ -413,6 +418,9 @@ void release(mot_attn* h) {
   if (!h) return;
   for (cudaEvent_t e : h->ev)
     if (e) cudaEventDestroy(e);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->side) cudaStreamDestroy(h->side);
   cudaFree(h->wo16);
   cudaFree(h->wqkv16);
   cudaFree(h->gamma);
@@ -426,22 +434,58 @@ void release(mot_attn* h) {
 // count and the optional per-launch events
 struct Launches {
   mot_attn* h;
-  cudaStream_t st;
+  cudaStream_t st;   // the caller's stream
+  cudaStream_t cur;  // where the next launch goes: st, or the handle's side stream
   int count = 0;
   int stage = 0;
+  int nev = 0;
+  bool side_pending = false;  // side-stream work not yet joined into st
+  cudaEvent_t last[2] = {};   // latest profiling event on st / on the side stream
   cudaError_t err = cudaSuccess;
-  Launches(mot_attn* handle, cudaStream_t s) : h(handle), st(s) {
-    if (h->profile) cudaEventRecord(h->ev[0], st);
+  Launches(mot_attn* handle, cudaStream_t s) : h(handle), st(s), cur(s) {
+    if (h->profile) last[0] = mark(st);
+  }
+  // every return path leaves st ordered after the side stream's work
+  ~Launches() {
+    if (side_pending) join();
+  }
+  void note(cudaError_t e) {
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+  }
+  cudaEvent_t mark(cudaStream_t s) {
+    if (nev >= static_cast<int>(sizeof(h->ev) / sizeof(h->ev[0]))) return nullptr;
+    cudaEvent_t e = h->ev[nev++];
+    cudaEventRecord(e, s);
+    return e;
+  }
+  // later launches go to the side stream, after all work issued so far on st
+  void fork() {
+    note(cudaEventRecord(h->ev_fork, st));
+    note(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+    cur = h->side;
+    side_pending = true;
+    if (h->profile) last[1] = mark(h->side);
+  }
+  void to_main() { cur = st; }
+  // st waits for all work issued on the side stream
+  void join() {
+    note(cudaEventRecord(h->ev_join, h->side));
+    note(cudaStreamWaitEvent(st, h->ev_join, 0));
+    cur = st;
+    side_pending = false;
   }
   void done(cudaError_t e) {
-    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    note(e);
     if (h->profile && count < kMaxStages) {
+      const int k = cur == st ? 0 : 1;
       h->stage_ids[count] = stage;
-      cudaEventRecord(h->ev[count + 1], st);
+      h->stage_start[count] = last[k];
+      last[k] = h->stage_end[count] = mark(cur);
     }
     ++count;
   }
   mot_status finish() {
+    if (side_pending) join();
     h->last_launches = count;
     h->stage_count = std::min(count, kMaxStages);
     return err == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
@@ -516,8 +560,11 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
             cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
   if (ok && cfg->enable_backward)
     ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess &&
-         cudaMalloc(&h->split_cnt, kSplitCounters * sizeof(int)) == cudaSuccess &&
-         cudaMemset(h->split_cnt, 0, kSplitCounters * sizeof(int)) == cudaSuccess;
+         cudaMalloc(&h->split_cnt, 2 * kSplitCounters * sizeof(int)) == cudaSuccess &&
+         cudaMemset(h->split_cnt, 0, 2 * kSplitCounters * sizeof(int)) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
     release(h);
     return MOT_ERR_CUDA;
@@ -823,7 +870,10 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
   __nv_bfloat16* g_hi = reinterpret_cast<__nv_bfloat16*>(ws + L.b_ghi);
   __nv_bfloat16* g_lo = reinterpret_cast<__nv_bfloat16*>(ws + L.b_glo);
   __half* b16 = reinterpret_cast<__half*>(ws + L.b_bqkv16);  // B_q|B_k|B_v in f16
+  // split-K partials and counters: one set for the caller's stream, one for the side stream
   void* split_ws = ws + L.b_split;
+  void* split_ws_side = ws + L.b_split + kSplitWsBytes;
+  int* split_cnt_side = h->split_cnt + kSplitCounters;
 
   const int Hq = c.n_q_heads, Hkv = c.n_kv_heads, d = c.hidden, M = L.M, RP = h->RP;
   const int qd = Hq * 128, kvd = Hkv * 128, nqkv = qd + 2 * kvd;
@@ -883,6 +933,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     lz.done(launch_gemm2<256, 6, EpiDattn>(core, ep, h->num_sms, st));
   }
   if (r > 0) {
+    // dB_o and dA_o feed nothing later in this call: side stream
+    lz.fork();
     // dB_o = dy^T u_o   [d, r], with u_o as its bf16 hi + lo pair
     lz.stage = ST_BWD_DB_O;
     {
@@ -898,8 +950,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.out32 = d_b[3];
       ep.ld32 = r;
       ep.accumulate32 = accumulate;
-      enable_split(core, split_ws, h->split_cnt);
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+      enable_split(core, split_ws_side, split_cnt_side);
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
     }
     // dA_o = (s g_o)^T o   [r, qd], computed as its transpose o^T (s g_o)
     lz.stage = ST_BWD_DA_O;
@@ -915,10 +967,11 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.ld32 = qd;
       ep.accumulate32 = accumulate;
       ep.transpose32 = 1;
-      enable_split(core, split_ws, h->split_cnt);
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+      enable_split(core, split_ws_side, split_cnt_side);
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
     }
   }
+  lz.to_main();
   // attention backward: dq^ over all keys, dk^, dv over the self keys
   {
     AttnBwdParams ap{};
@@ -981,6 +1034,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       enable_split(core, split_ws, h->split_cnt);
       lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
     }
+    // dB_j and dA_j feed nothing later in this call: side stream
+    lz.fork();
     for (int j = 0; j < 3; ++j) {
       // dB_j = d{q,k,v}_pre^T u_j   [out_j, r]
       lz.stage = ST_BWD_DB_QKV;
@@ -995,8 +1050,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.out32 = d_b[j];
       ep.ld32 = r;
       ep.accumulate32 = accumulate;
-      enable_split(core, split_ws, h->split_cnt);
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
+      enable_split(core, split_ws_side, split_cnt_side);
+      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
     }
     {
       // dA_j = (s g_j)^T x for the three projections in one GEMM over x^T,
@@ -1018,9 +1073,10 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.M = d;
       ep.transpose = 1;
       ep.accumulate = accumulate;
-      enable_split(core, split_ws, h->split_cnt);
-      lz.done(launch_gemm_narrow<EpiLoraGrad>(RP, core, ep, h->num_sms, st));
+      enable_split(core, split_ws_side, split_cnt_side);
+      lz.done(launch_gemm_narrow<EpiLoraGrad>(RP, core, ep, h->num_sms, lz.cur));
     }
+    lz.to_main();
   }
   // dx = dq W_q + dk W_k + dv W_v + sum_j ((s g_j)_hi + (s g_j)_lo) A_j
   lz.stage = ST_BWD_DX;
@@ -1200,10 +1256,12 @@ mot_status mot_dev_stage_times(mot_attn_t h, int32_t* ids, float* ms, int32_t ma
   if (!h->profile) return MOT_ERR_INVALID_ARGUMENT;
   *count = h->stage_count;
   if (h->stage_count == 0) return MOT_OK;
-  if (cudaEventSynchronize(h->ev[h->stage_count]) != cudaSuccess) return MOT_ERR_CUDA;
   for (int i = 0; i < h->stage_count && i < max; ++i) {
     ids[i] = h->stage_ids[i];
-    if (cudaEventElapsedTime(&ms[i], h->ev[i], h->ev[i + 1]) != cudaSuccess) return MOT_ERR_CUDA;
+    if (!h->stage_start[i] || !h->stage_end[i]) return MOT_ERR_CUDA;
+    if (cudaEventSynchronize(h->stage_end[i]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms[i], h->stage_start[i], h->stage_end[i]) != cudaSuccess)
+      return MOT_ERR_CUDA;
   }
   return MOT_OK;
 }
