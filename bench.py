@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the 2048^2 CFG workload, keyed by the sha256 of the
 # kernel's source file at capture time: a changed kernel reports null.
 TRAFFIC = {
-    "attn_fwd": {"sha256": "455925fac2614ce6a7ded279b5b33f1c00db2d54c4046cd29f681133c7fc33b2",
-                 "bytes": 104929024 + 32312832},
+    "attn_fwd": {"sha256": "fa113b24ee3a31c44f97f0d625781be083da09732a26b1f2e7bfacc173b8f602",
+                 "bytes": 104928256 + 32443136},
     "qkv_gemm": {"sha256": "a3e27cc7e03cf01608307002321cef734c2a77a5a52b7c90a6c75e27712b49b3",
                  "bytes": 249139456 + 81316096},
 }
