@@ -37,18 +37,24 @@ constexpr uint32_t kMnBoxBytes = 64 * 64 * 2;  // MN-major TMA box: 64 MN x 64 K
 // TMA boxes and described to the tensor core as transposed operands.
 struct GemmSeg {
   int a_map;
-  int a_k0[kMaxRegions];   // per N-region (the LoRA extension reads a different u slice per region)
-  int b_map[kMaxRegions];  // per N-region B tensor
+  int a_k0[kMaxRegions];   // per region (the LoRA extension reads a different u slice per region)
+  int b_map[kMaxRegions];  // per region B tensor
   int b_k0;
   int kb;
   uint32_t idesc;
   int a_mn, b_mn;
+  // dual (1-CTA kernel instantiated with kDual): every k-block also loads a
+  // second B tile from b2_map and both products accumulate into D, so the A
+  // tile is read once for two B operands (a bf16 hi + lo pair)
+  int dual;
+  int b2_map[kMaxRegions];
 };
 
 struct GemmCore {
   CUtensorMap maps[kMaxMaps];
   int region_n0[kMaxRegions + 1];  // region i covers D columns [region_n0[i], region_n0[i+1])
   int num_regions;
+  int regions_on_m;  // 1-CTA kernel: regions split D rows instead (region_n0 then holds row bounds)
   GemmSeg segs[kMaxSegs];
   int num_segs;
   int M, N;
@@ -95,24 +101,25 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
   return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool kDual = false>
 struct GemmSmem {
   static constexpr uint32_t kABytes = kBM * kBK * 2;
-  static constexpr uint32_t kBBytes = BN * kBK * 2;
-  static constexpr uint32_t kBarOffset = STAGES * (kABytes + kBBytes);
+  static constexpr uint32_t kBBytes = BN * kBK * 2;                  // one B tile
+  static constexpr uint32_t kBStage = kDual ? 2 * kBBytes : kBBytes;  // B tiles of a stage
+  static constexpr uint32_t kBarOffset = STAGES * (kABytes + kBStage);
   static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
 };
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, class Epi, bool kDual = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmArgs<Epi> args) {
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128, whole 64-column boxes");
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, kDual>;
   constexpr uint32_t kTmemCols = tmem_cols_for(2 * BN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * L::kABytes;
+  uint8_t* sB = smem + STAGES * L::kABytes;  // stage s: B tile(s) at s * kBStage
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -153,6 +160,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const WaitGuard wg{abort_flag, g.status};
 
   const int num_tiles = g.tiles_m * g.tiles_n;
+  const bool rows_reg = g.regions_on_m != 0;
   const int splits = g.k_splits > 1 ? g.k_splits : 1;
   const int num_items = num_tiles * splits;
   const int total_kb = g.total_kb;
@@ -172,32 +180,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
         const int m0 = tm * kBM, n0 = tn * BN;
-        const int reg0 = region_of(g, n0);
+        const int reg0 = region_of(g, rows_reg ? m0 : n0);
         int gk = 0;  // k-blocks of the segments before this one
         for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
           const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb, a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
           const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);
           gk += nkb;
+          const bool dual = kDual && sg.dual;
           const CUtensorMap* amap = &g.maps[sg.a_map];
           // B boxes of this tile: up to 4 (map, row/column offset) pairs
           const int box_n = b_mn ? 64 : b_box_rows;
           const int nbox = BN / box_n;
           const CUtensorMap* bmap[4];
+          const CUtensorMap* bmap2[4];
           int bcoord[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int n = n0 + (i < nbox ? i : 0) * box_n;
-            const int r = region_of(g, n);
+            const int r = rows_reg ? reg0 : region_of(g, n);
             bmap[i] = &g.maps[sg.b_map[r]];
-            bcoord[i] = n - g.region_n0[r];
+            bmap2[i] = &g.maps[sg.b2_map[r]];
+            bcoord[i] = rows_reg ? n : n - g.region_n0[r];
           }
           const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
           for (int kb = kb0; kb < kb1; ++kb) {
             mbar_wait(&empty[stage], phase ^ 1u, wg);
-            mbar_expect_tx(&full[stage], L::kABytes + L::kBBytes);
+            mbar_expect_tx(&full[stage], L::kABytes + (dual ? 2 : 1) * L::kBBytes);
             uint8_t* a_dst = sA + stage * L::kABytes;
-            uint8_t* b_dst = sB + stage * L::kBBytes;
+            uint8_t* b_dst = sB + stage * L::kBStage;
             const int ka = a_k0 + kb * kBK, kbk = b_k0 + kb * kBK;
             if (a_mn) {
               tma_load_2d(a_dst, amap, &full[stage], m0, ka);
@@ -212,6 +223,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 tma_load_2d(b_dst + i * box_bytes, bmap[i], &full[stage], bcoord[i], kbk);
               else
                 tma_load_2d(b_dst + i * box_bytes, bmap[i], &full[stage], kbk, bcoord[i]);
+            }
+            if (dual) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                if (i >= nbox) break;
+                uint8_t* d2 = b_dst + L::kBBytes + i * box_bytes;
+                if (b_mn)
+                  tma_load_2d(d2, bmap2[i], &full[stage], bcoord[i], kbk);
+                else
+                  tma_load_2d(d2, bmap2[i], &full[stage], kbk, bcoord[i]);
+              }
             }
             if (++stage == STAGES) {
               stage = 0;
@@ -239,19 +261,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const GemmSeg& sg = g.segs[si];
           const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb;
           const uint32_t idesc = sg.idesc;
+          const bool dual = kDual && sg.dual;
           const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);
           gk += nkb;
           for (int kb = kb0; kb < kb1; ++kb) {
             mbar_wait(&full[stage], phase, wg);
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA + stage * L::kABytes);
-            const uint32_t b_addr = smem_u32(sB + stage * L::kBBytes);
+            const uint32_t b_addr = smem_u32(sB + stage * L::kBStage);
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t ad = a_mn ? mnmajor_desc(a_addr, kk, kMnBoxBytes) : kmajor_desc(a_addr, kk, L::kABytes);
               const uint64_t bd = b_mn ? mnmajor_desc(b_addr, kk, kMnBoxBytes) : kmajor_desc(b_addr, kk, L::kBBytes);
               umma_ss(d_tmem, ad, bd, idesc, accumulate);
               accumulate = 1u;
+              if (dual) {
+                const uint32_t b2 = b_addr + L::kBBytes;
+                const uint64_t bd2 = b_mn ? mnmajor_desc(b2, kk, kMnBoxBytes) : kmajor_desc(b2, kk, L::kBBytes);
+                umma_ss(d_tmem, ad, bd2, idesc, 1u);
+              }
             }
             umma_commit(&empty[stage]);
             if (++stage == STAGES) {
@@ -307,12 +335,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             float v[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            // in split order; two splits' loads in flight at a time
+            int sp = 0;
 #pragma unroll 1
-            for (int sp = 0; sp < splits; ++sp) {
-              const float4* q = base + static_cast<long long>(sp) * (BN / 4) * kBM + (c >> 2) * kBM;
+            for (; sp + 1 < splits; sp += 2) {
+              const float4* q0 = base + static_cast<long long>(sp) * (BN / 4) * kBM + (c >> 2) * kBM;
+              const float4* q1 = q0 + (BN / 4) * kBM;
+              float4 f0[8], f1[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float4 f = __ldcg(q + i * kBM);
+                f0[i] = __ldcg(q0 + i * kBM);
+                f1[i] = __ldcg(q1 + i * kBM);
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                v[4 * i] = (v[4 * i] + f0[i].x) + f1[i].x;
+                v[4 * i + 1] = (v[4 * i + 1] + f0[i].y) + f1[i].y;
+                v[4 * i + 2] = (v[4 * i + 2] + f0[i].z) + f1[i].z;
+                v[4 * i + 3] = (v[4 * i + 3] + f0[i].w) + f1[i].w;
+              }
+            }
+            if (sp < splits) {
+              const float4* q0 = base + static_cast<long long>(sp) * (BN / 4) * kBM + (c >> 2) * kBM;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 f = __ldcg(q0 + i * kBM);
                 v[4 * i] += f.x;
                 v[4 * i + 1] += f.y;
                 v[4 * i + 2] += f.z;
@@ -634,37 +681,33 @@ struct EpiStore {
       for (int i = 0; i < 3; ++i)
         if (p.o16[i].ptr) store16(p, i, m, n, v, ncols, overflow);
       if (p.out32) {
+        // every old value is loaded before the first store, so the loads
+        // overlap instead of each waiting for the store before it
         if (p.transpose32) {
+          float old[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (k >= ncols) continue;
-            float* o = p.out32 + static_cast<long long>(n + k) * p.ld32 + m;
-            const float w = v[k] * p.scale32;
-            *o = p.accumulate32 ? *o + w : w;
-          }
+          for (int k = 0; k < 32; ++k)
+            old[k] = (p.accumulate32 && k < ncols) ? p.out32[static_cast<long long>(n + k) * p.ld32 + m] : 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k < ncols) p.out32[static_cast<long long>(n + k) * p.ld32 + m] = fmaf(v[k], p.scale32, old[k]);
         } else if (ncols == 32) {
           float4* dst = reinterpret_cast<float4*>(p.out32 + m * p.ld32 + n);
+          float4 old[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 w = make_float4(v[4 * i] * p.scale32, v[4 * i + 1] * p.scale32, v[4 * i + 2] * p.scale32,
-                                   v[4 * i + 3] * p.scale32);
-            if (p.accumulate32) {
-              const float4 o = dst[i];
-              w.x += o.x;
-              w.y += o.y;
-              w.z += o.z;
-              w.w += o.w;
-            }
-            dst[i] = w;
-          }
+          for (int i = 0; i < 8; ++i) old[i] = p.accumulate32 ? dst[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(fmaf(v[4 * i], p.scale32, old[i].x), fmaf(v[4 * i + 1], p.scale32, old[i].y),
+                                 fmaf(v[4 * i + 2], p.scale32, old[i].z), fmaf(v[4 * i + 3], p.scale32, old[i].w));
         } else {
+          float* o = p.out32 + m * p.ld32 + n;
+          float old[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (k >= ncols) continue;
-            float* o = p.out32 + m * p.ld32 + n + k;
-            const float w = v[k] * p.scale32;
-            *o = p.accumulate32 ? *o + w : w;
-          }
+          for (int k = 0; k < 32; ++k) old[k] = (p.accumulate32 && k < ncols) ? o[k] : 0.f;
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (k < ncols) o[k] = fmaf(v[k], p.scale32, old[k]);
         }
       }
     }
@@ -692,14 +735,53 @@ struct EpiLoraGrad {
       float v[32];
       load_row32(taddr + c, v);
       if (m >= p.M) continue;
+      // old values first (independent loads), then the stores
+      float* dst[32];
+      float old[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int n = n0 + c + i;
         const int j = n / p.RP, k = n - j * p.RP;
-        if (j > 2 || k >= p.r) continue;
-        float* o = p.transpose ? p.out[j] + static_cast<long long>(k) * p.ld + m : p.out[j] + m * p.ld + k;
-        *o = p.accumulate ? *o + v[i] : v[i];
+        dst[i] = (j > 2 || k >= p.r) ? nullptr
+                 : p.transpose       ? p.out[j] + static_cast<long long>(k) * p.ld + m
+                                     : p.out[j] + m * p.ld + k;
+        old[i] = (p.accumulate && dst[i]) ? *dst[i] : 0.f;
       }
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (dst[i]) *dst[i] = old[i] + v[i];
+    }
+  }
+};
+
+// D rows [row0[j], row0[j+1]) (j < 3) go to out[j], row m - row0[j], the
+// first `cols` columns, row-major with leading dimension ld; accumulate adds
+// into what is there (the three LoRA-up gradients of q, k, v in one GEMM).
+struct EpiRowBlocks {
+  struct Params {
+    float* out[3];
+    int row0[4];
+    long long ld;
+    int cols;
+    int accumulate;
+  };
+  template <int BN>
+  __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
+                                               int* status) {
+    const int m = m0 + row;
+    const int j = (m >= p.row0[1]) + (m >= p.row0[2]);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      load_row32(taddr + c, v);
+      if (m >= p.row0[3]) continue;
+      float* o = p.out[j] + static_cast<long long>(m - p.row0[j]) * p.ld;
+      float old[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) old[i] = (p.accumulate && n0 + c + i < p.cols) ? o[n0 + c + i] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + c + i < p.cols) o[n0 + c + i] = old[i] + v[i];
     }
   }
 };
@@ -733,9 +815,12 @@ struct EpiDattn {
         const long long off = static_cast<long long>(m) * p.Hq * 128 + head * 128 + c * 32;
         const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
         uint4* d4 = reinterpret_cast<uint4*>(p.dout + off);
+        uint4 ow4[4];  // loaded ahead of the dO stores
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ow4[i] = o4[i];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint4 ow = o4[i];
+          const uint4 ow = ow4[i];
           const __half2* oh = reinterpret_cast<const __half2*>(&ow);
           uint32_t w[4];
 #pragma unroll

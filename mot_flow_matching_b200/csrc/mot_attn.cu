@@ -197,6 +197,12 @@ int pick_splits(int tiles, int total_kb, int num_sms, int bn) {
   return best;
 }
 
+// second B operand of a dual segment (same box coordinates, map b2 in every region)
+void set_dual(GemmSeg& sg, int b2) {
+  sg.dual = 1;
+  for (int i = 0; i < kMaxRegions; ++i) sg.b2_map[i] = b2;
+}
+
 // let launch_gemm split K (1-CTA kernel; partials in ws, counters in cnt)
 void enable_split(GemmCore& c, void* ws, int* cnt) {
   c.k_splits = -1;
@@ -204,12 +210,12 @@ void enable_split(GemmCore& c, void* ws, int* cnt) {
   c.split_cnt = cnt;
 }
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, class Epi, bool kDual = false>
 cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, int num_sms, cudaStream_t st) {
   static_assert(sizeof(GemmArgs<Epi>) <= 4096, "kernel parameter block");
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, kDual>;
   static_assert(L::kBytes <= 232448, "shared memory");
-  auto kern = gemm_kernel<BN, STAGES, Epi>;
+  auto kern = gemm_kernel<BN, STAGES, Epi, kDual>;
   static std::once_flag once;
   std::call_once(once, [&] { set_smem_attr(kern, L::kBytes); });
   GemmArgs<Epi> args;
@@ -227,6 +233,16 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   return cudaGetLastError();
 }
 
+// CTA pairs a pair-kernel launch of `tiles` tiles uses: the fewest that
+// finish in the same number of rounds of tiles as all SMs would, so every
+// pair gets the same tile count and the SMs left over can run other work
+// (the backward's side-stream GEMMs) for the whole duration
+int pair_count(int tiles, int num_sms) {
+  const int max_pairs = std::max(1, num_sms / 2);
+  const int rounds = (tiles + max_pairs - 1) / max_pairs;
+  return std::max(1, (tiles + rounds - 1) / rounds);
+}
+
 // 2-SM (CTA pair) launch: core.tiles_m counts 256-row tiles
 template <int BN, int STAGES, class Epi>
 cudaError_t launch_gemm2(const GemmCore& core, const typename Epi::Params& ep, int num_sms, cudaStream_t st) {
@@ -239,8 +255,10 @@ cudaError_t launch_gemm2(const GemmCore& core, const typename Epi::Params& ep, i
   GemmArgs<Epi> args;
   args.core = core;
   args.epi = ep;
-  const int tiles = core.tiles_m * core.tiles_n;
-  const int pairs = std::max(1, std::min(tiles, num_sms / 2));
+  // the fewest pairs that finish in the same number of rounds of tiles: every
+  // pair gets the same tile count, and the SMs left over can run other work
+  // (the backward's side-stream GEMMs) for the whole duration
+  const int pairs = pair_count(core.tiles_m * core.tiles_n, num_sms);
   kern<<<2 * pairs, kGemmThreads, L::kBytes, st>>>(args);
   return cudaGetLastError();
 }
@@ -253,6 +271,15 @@ template <class Epi>
 cudaError_t launch_gemm_narrow(int BN, const GemmCore& core, const typename Epi::Params& ep, int num_sms,
                                cudaStream_t st) {
   return BN == 64 ? launch_gemm<64, 8, Epi>(core, ep, num_sms, st) : launch_gemm<128, 6, Epi>(core, ep, num_sms, st);
+}
+
+// the same with dual (hi + lo) B segments; BN = 64, 128 or 192
+template <class Epi>
+cudaError_t launch_gemm_dual(int BN, const GemmCore& core, const typename Epi::Params& ep, int num_sms,
+                             cudaStream_t st) {
+  if (BN == 64) return launch_gemm<64, 6, Epi, true>(core, ep, num_sms, st);
+  if (BN == 128) return launch_gemm<128, 4, Epi, true>(core, ep, num_sms, st);
+  return launch_gemm<192, 3, Epi, true>(core, ep, num_sms, st);
 }
 
 void core_init(GemmCore& c, int M, int N, int BN, int b_box_rows, int* status) {
@@ -944,14 +971,14 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
           !map2d_mn(&core.maps[3], u_olo, true, RP, M, RP))
         return MOT_ERR_CUDA;
       core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
-      core.segs[1] = seg1(0, 0, 3, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
-      core.num_segs = 2;
+      set_dual(core.segs[0], 3);
+      core.num_segs = 1;
       EpiStore::Params ep = store_params(d, r);
       ep.out32 = d_b[3];
       ep.ld32 = r;
       ep.accumulate32 = accumulate;
       enable_split(core, split_ws_side, split_cnt_side);
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
+      lz.done(launch_gemm_dual<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
     }
     // dA_o = (s g_o)^T o   [r, qd], computed as its transpose o^T (s g_o)
     lz.stage = ST_BWD_DA_O;
@@ -1036,35 +1063,49 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     }
     // dB_j and dA_j feed nothing later in this call: side stream
     lz.fork();
-    for (int j = 0; j < 3; ++j) {
-      // dB_j = d{q,k,v}_pre^T u_j   [out_j, r]
+    {
+      // dB_j = d{q,k,v}_pre^T u_j   [out_j, r] for the three projections in
+      // one GEMM: D rows are the nqkv columns of d{q,k,v}_pre, and row block j
+      // (a whole number of 128-row tiles) meets u_j
       lz.stage = ST_BWD_DB_QKV;
       GemmCore core;
-      core_init(core, outj[j], RP, RP, RP, h->status);
-      if (!map2d_mn(&core.maps[0], dqkv + col0[j], false, outj[j], M, nqkv) ||
-          !map2d_mn(&core.maps[2], u_qkv + j * RP, false, RP, M, 3 * RP))
-        return MOT_ERR_CUDA;
+      core_init(core, nqkv, RP, RP, RP, h->status);
+      if (!map2d_mn(&core.maps[0], dqkv, false, nqkv, M, nqkv)) return MOT_ERR_CUDA;
+      for (int j = 0; j < 3; ++j)
+        if (!map2d_mn(&core.maps[2 + j], u_qkv + j * RP, false, RP, M, 3 * RP)) return MOT_ERR_CUDA;
+      core.regions_on_m = 1;
+      core.num_regions = 3;
+      for (int j = 0; j < 3; ++j) core.region_n0[j] = col0[j];
+      core.region_n0[3] = nqkv;
       core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, false, false, true, true), true, true);
+      for (int j = 0; j < 3; ++j) core.segs[0].b_map[j] = 2 + j;
       core.num_segs = 1;
-      EpiStore::Params ep = store_params(outj[j], r);
-      ep.out32 = d_b[j];
-      ep.ld32 = r;
-      ep.accumulate32 = accumulate;
+      EpiRowBlocks::Params ep{};
+      for (int j = 0; j < 3; ++j) {
+        ep.out[j] = d_b[j];
+        ep.row0[j] = col0[j];
+      }
+      ep.row0[3] = nqkv;
+      ep.ld = r;
+      ep.cols = r;
+      ep.accumulate = accumulate;
       enable_split(core, split_ws_side, split_cnt_side);
-      lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, lz.cur));
+      lz.done(launch_gemm_narrow<EpiRowBlocks>(RP, core, ep, h->num_sms, lz.cur));
     }
     {
       // dA_j = (s g_j)^T x for the three projections in one GEMM over x^T,
       // with (s g_j) as its bf16 hi + lo pair; block j goes to dA_j transposed
       lz.stage = ST_BWD_DA_QKV;
       GemmCore core;
-      core_init(core, d, 3 * RP, RP, RP, h->status);
+      // one 3 RP-wide tile when it fits the MMA (x^T read once), else RP-wide
+      const int bn = 3 * RP <= 256 ? 3 * RP : RP;
+      core_init(core, d, 3 * RP, bn, RP, h->status);
       if (!map2d_mn(&core.maps[0], x, true, d, M, d) || !map2d_mn(&core.maps[2], g_hi, true, 3 * RP, M, 3 * RP) ||
           !map2d_mn(&core.maps[3], g_lo, true, 3 * RP, M, 3 * RP))
         return MOT_ERR_CUDA;
-      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
-      core.segs[1] = seg1(0, 0, 3, kb_tok, idesc_f16(128, RP, true, true, true, true), true, true);
-      core.num_segs = 2;
+      core.segs[0] = seg1(0, 0, 2, kb_tok, idesc_f16(128, bn, true, true, true, true), true, true);
+      set_dual(core.segs[0], 3);
+      core.num_segs = 1;
       EpiLoraGrad::Params ep{};
       for (int j = 0; j < 3; ++j) ep.out[j] = d_a[j];
       ep.ld = d;
@@ -1074,7 +1115,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ep.transpose = 1;
       ep.accumulate = accumulate;
       enable_split(core, split_ws_side, split_cnt_side);
-      lz.done(launch_gemm_narrow<EpiLoraGrad>(RP, core, ep, h->num_sms, lz.cur));
+      lz.done(launch_gemm_dual<EpiLoraGrad>(bn, core, ep, h->num_sms, lz.cur));
     }
     lz.to_main();
   }
