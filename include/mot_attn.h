@@ -111,7 +111,12 @@ mot_status mot_attn_query_sizes(const mot_attn_config* cfg, int32_t batch, int32
 /* Create a handle. Validates cfg (host) and the weight pointers, allocates
  * the handle's own device copies (f16 w_o, f32 norm gains, f32 RoPE cos/sin
  * table built in fp64 on the host for positions < max_prefix +
- * max_img_tokens) and enqueues their initialisation on `stream`.
+ * max_img_tokens) and enqueues their initialisation on `stream`. It also
+ * allocates the split-K scratch of the LoRA-down GEMMs (f32 partial tiles
+ * for up to max_batch * max_img_tokens rows, at most 32 MiB, when
+ * lora_rank > 0) with its arrival counters, and, with enable_backward, an
+ * f16 copy of w_q|w_k|w_v and a second stream plus two events on which the
+ * backward runs the LoRA-gradient GEMMs that feed nothing later in the call.
  * Returns MOT_OK and *out, or an error and *out = NULL. */
 mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* weights,
                            void* stream, mot_attn_t* out);
@@ -144,7 +149,11 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t batch, int32_t 
  *   d_a[4], d_b[4]  device f32, q,k,v,o order, shapes of a_* / b_*;
  *            accumulate != 0 adds into their contents, else overwrites.
  *            All NULL is allowed when lora_rank == 0.
- * Requires cfg.enable_backward. Deterministic: same inputs, same bits. */
+ * Requires cfg.enable_backward. Deterministic: same inputs, same bits.
+ * Part of the work (the dB and dA GEMMs) runs on the handle's own stream,
+ * which waits for `stream` where its inputs are produced; before returning,
+ * the call makes `stream` wait for that work, so everything the call writes
+ * is ordered before later work on `stream`, as if it all ran there. */
 mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_t batch,
                              int32_t img_tokens, const void* k_cache, const void* v_cache,
                              const int32_t* prefix_len, int32_t prefix_max, const void* saved,

@@ -70,6 +70,7 @@ struct GemmCore {
   int total_kb;
   float4* split_ws;  // [tiles * k_splits][BN / 4][128]
   int* split_cnt;    // [tiles], zero between launches
+  size_t split_cap;  // bytes at split_ws (host side: bounds the split count)
 };
 
 template <class Epi>

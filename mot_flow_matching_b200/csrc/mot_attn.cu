@@ -183,11 +183,11 @@ void set_smem_attr(K kernel, size_t bytes) {
 // fewest splits that come close to the best SM balance ceil(items/SMs)/S,
 // each split costing a little for its partial-tile round trip; at most 16,
 // at least two k-blocks per split, partials within the split workspace.
-int pick_splits(int tiles, int total_kb, int num_sms, int bn) {
+int pick_splits(int tiles, int total_kb, int num_sms, int bn, size_t cap_bytes) {
   int best = 1;
   double best_cost = static_cast<double>((tiles + num_sms - 1) / num_sms);
   for (int sp = 2; sp <= 16 && 2 * sp <= total_kb; ++sp) {
-    if (static_cast<size_t>(tiles) * sp * bn * kBM * 4 > kSplitWsBytes) break;
+    if (static_cast<size_t>(tiles) * sp * bn * kBM * 4 > cap_bytes) break;
     const double cost = static_cast<double>((tiles * sp + num_sms - 1) / num_sms) / sp + 0.02 * (sp - 1);
     if (cost < best_cost - 1e-9) {
       best = sp;
@@ -203,11 +203,12 @@ void set_dual(GemmSeg& sg, int b2) {
   for (int i = 0; i < kMaxRegions; ++i) sg.b2_map[i] = b2;
 }
 
-// let launch_gemm split K (1-CTA kernel; partials in ws, counters in cnt)
-void enable_split(GemmCore& c, void* ws, int* cnt) {
+// let launch_gemm split K (1-CTA kernel; partials in ws of cap bytes, counters in cnt)
+void enable_split(GemmCore& c, void* ws, int* cnt, size_t cap = kSplitWsBytes) {
   c.k_splits = -1;
   c.split_ws = static_cast<float4*>(ws);
   c.split_cnt = cnt;
+  c.split_cap = cap;
 }
 
 template <int BN, int STAGES, class Epi, bool kDual = false>
@@ -226,7 +227,7 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   for (int i = 0; i < core.num_segs; ++i) total_kb += core.segs[i].kb;
   args.core.total_kb = total_kb;
   args.core.k_splits =
-      core.k_splits < 0 && tiles <= kSplitCounters ? pick_splits(tiles, total_kb, num_sms, BN) : 1;
+      core.k_splits < 0 && tiles <= kSplitCounters ? pick_splits(tiles, total_kb, num_sms, BN, core.split_cap) : 1;
   const int items = tiles * args.core.k_splits;
   const int grid = std::max(1, std::min(items, num_sms));
   kern<<<grid, kGemmThreads, L::kBytes, st>>>(args);
@@ -369,7 +370,9 @@ struct mot_attn {
   float2* rope = nullptr;
   int rope_len = 0;
   int* status = nullptr;
-  int* split_cnt = nullptr;  // [2][kSplitCounters] split-K arrival counters (backward; caller's / side stream)
+  int* split_cnt = nullptr;  // [3][kSplitCounters] split-K arrival counters: backward (caller's / side stream), forward
+  void* fsplit = nullptr;    // forward split-K partials (LoRA down), sized for max_batch x max_img_tokens
+  size_t fsplit_bytes = 0;
   int num_sms = 148;
   int last_launches = 0;
   // backward: a second stream for the gradient GEMMs nothing later depends on
@@ -454,6 +457,7 @@ void release(mot_attn* h) {
   cudaFree(h->rope);
   cudaFree(h->status);
   cudaFree(h->split_cnt);
+  cudaFree(h->fsplit);
   delete h;
 }
 
@@ -585,10 +589,17 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
   bool ok = cudaMalloc(&h->wo16, d * qd * 2) == cudaSuccess && cudaMalloc(&h->gamma, 2 * dh * 4) == cudaSuccess &&
             cudaMalloc(&h->rope, static_cast<size_t>(h->rope_len) * 64 * sizeof(float2)) == cudaSuccess &&
             cudaMalloc(&h->status, sizeof(int)) == cudaSuccess;
+  ok = ok && cudaMalloc(&h->split_cnt, 3 * kSplitCounters * sizeof(int)) == cudaSuccess &&
+       cudaMemset(h->split_cnt, 0, 3 * kSplitCounters * sizeof(int)) == cudaSuccess;
+  if (ok && cfg->lora_rank > 0) {
+    // the forward LoRA-down GEMMs' split-K partials: up to 4 splits of the
+    // 128-row tiles of the largest call, 192 (or 128) f32 columns each
+    const size_t tiles = (static_cast<size_t>(cfg->max_batch) * cfg->max_img_tokens + kBM - 1) / kBM;
+    h->fsplit_bytes = std::min(kSplitWsBytes * 2, tiles * 4 * 192 * kBM * 4);
+    ok = cudaMalloc(&h->fsplit, h->fsplit_bytes) == cudaSuccess;
+  }
   if (ok && cfg->enable_backward)
     ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess &&
-         cudaMalloc(&h->split_cnt, 2 * kSplitCounters * sizeof(int)) == cudaSuccess &&
-         cudaMemset(h->split_cnt, 0, 2 * kSplitCounters * sizeof(int)) == cudaSuccess &&
          cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess &&
          cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
@@ -726,6 +737,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     EpiStore::Params ep = store_params(M, 3 * RP);
     set_out16(ep, 0, u_qkv, 3 * RP, false, h->scale);
     ep.check_f16 = 1;
+    enable_split(core, h->fsplit, h->split_cnt + 2 * kSplitCounters, h->fsplit_bytes);
     if (BN == 192)
       lz.done(launch_gemm<192, 5, EpiStore>(core, ep, h->num_sms, st));
     else
@@ -819,6 +831,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
       set_out16(ep, 2, u_olo, RP, true, 1.0f, 1);
     }
     ep.check_f16 = 1;
+    enable_split(core, h->fsplit, h->split_cnt + 2 * kSplitCounters, h->fsplit_bytes);
     lz.done(launch_gemm_narrow<EpiStore>(RP, core, ep, h->num_sms, st));
   }
   // 7. O projection (+ LoRA up): y bf16 and optional f32
