@@ -168,13 +168,6 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
-
-
 def oracle_sample(wl, inputs_cpu, rows_per_branch, seed=0):
     """One oracle forward restricted to `rows_per_branch` query rows per branch."""
     import numpy as np
@@ -198,7 +191,8 @@ def blas_threads():
 
 
 def run_reference(args):
-    world, rank, _ = dist_setup()
+    from mot_flow_matching_b200 import dp
+    world, rank, _ = dp.world_info()
     if rank != 0:
         return 0
     from mot_flow_matching_b200 import synth
@@ -272,7 +266,7 @@ def train_steps(bundle, dev, flush, stream, args, world):
     """Forward (activations kept) + backward of the training workload; each
     timed separately with CUDA events, per-launch times from the library."""
     import torch
-    import torch.distributed as dist
+    from mot_flow_matching_b200 import dp
     from mot_flow_matching_b200.layer import mot_dev_profile, mot_dev_stage_times
     wl, td, layer = bundle
     pl = [int(v) for v in td["prefix_len"]]
@@ -292,8 +286,7 @@ def train_steps(bundle, dev, flush, stream, args, world):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
     mot_dev_profile(layer.handle, True)
     fwd_ms, bwd_ms, stages, launches = [], [], {}, 0
     for _ in range(args.steps):
@@ -316,7 +309,8 @@ def train_steps(bundle, dev, flush, stream, args, world):
     mot_dev_profile(layer.handle, False)
     assert layer.device_status() == 0
     layer.close()
-    f, b = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    f = dp.max_over_ranks(statistics.mean(fwd_ms), world, dev)
+    b = dp.max_over_ranks(statistics.mean(bwd_ms), world, dev)
     fwd_flops = sum(stage_work(wl, n)[0] for n in ("lora_down_qkv", "qkv_gemm", "attn_fwd", "lora_down_o", "o_gemm"))
     bwd_flops = sum(stage_work(wl, n)[0] * (3 if n in ("bwd_g_qkv", "bwd_db_qkv", "bwd_da_qkv") else 1)
                     for n in stages if n.startswith(("bwd_", "attn_bwd")))
@@ -335,25 +329,23 @@ def train_steps(bundle, dev, flush, stream, args, world):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     from mot_flow_matching_b200 import build as build_mod
     from mot_flow_matching_b200 import synth
     from mot_flow_matching_b200.layer import MotAttnLayer, mot_dev_profile, mot_dev_stage_times
 
-    world, rank, local = dist_setup()
+    from mot_flow_matching_b200 import dp
+    world, rank, local = dp.world_info()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    dp.init_group(world, "nccl", dev)
     if rank == 0:
         build_mod.build()
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
 
+    # each rank: its own data shard (x, cache, dy), replicated weights
     def make(index):
         wl = synth.WORKLOADS[index]
-        t = synth.workload_inputs(index)
+        t = synth.workload_inputs(index, shard=rank)
         td = {k: (v.to(dev) if k != "prefix_len" else v) for k, v in t.items()}
         wts = {k: td[k] for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
                                   "b_q", "b_k", "b_v", "b_o") if k in td}
@@ -366,7 +358,7 @@ def run_ours(args):
 
     def make_train():
         wl = synth.WORKLOADS[TRAIN_INDEX]
-        t = synth.workload_inputs(TRAIN_INDEX)
+        t = synth.workload_inputs(TRAIN_INDEX, shard=rank)
         td = {k: (v.to(dev) if k != "prefix_len" else v) for k, v in t.items()}
         wts = {k: td[k] for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "a_k", "a_v", "a_o",
                                   "b_q", "b_k", "b_v", "b_o") if k in td}
@@ -383,8 +375,7 @@ def run_ours(args):
             layer.forward(x, kc, vc, pl, y=y, workspace=ws)
         torch.cuda.synchronize(dev)
         mot_dev_profile(layer.handle, profile)
-        if world > 1:
-            dist.barrier()
+        dp.barrier(world)
         torch.cuda.synchronize(dev)
         step_ms, stages = [], {}
         launches = 0
@@ -410,14 +401,10 @@ def run_ours(args):
     clocks.start()
     step_ms, stages, launches = device_steps(wl, td, layer, args.steps, args.warmup, True)
     clk = clocks.stop()
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = dp.max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     tokens = wl.batch * wl.img_tokens
-    value = world * tokens * args.steps / (total_ms / 1e3)
+    value = dp.aggregate_rate(tokens, args.steps, total_ms, world)
 
     # end to end through the public call with host buffers: pinned H2D of
     # x and the prefix cache, the layer, D2H of y, every step
@@ -440,8 +427,7 @@ def run_ours(args):
     for _ in range(max(3, args.warmup)):
         e2e_step()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    dp.barrier(world)
     e2e_ms = 0.0
     for _ in range(args.steps):
         flush.zero_()
@@ -452,11 +438,8 @@ def run_ours(args):
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = world * tokens * args.steps / (e2e_ms / 1e3)
+    e2e_ms = dp.max_over_ranks(e2e_ms, world, dev)
+    e2e_value = dp.aggregate_rate(tokens, args.steps, e2e_ms, world)
     h2d = (x_h.numel() + kc_h.numel() + vc_h.numel()) * 2
     d2h = y_h.numel() * 2
 
@@ -470,8 +453,9 @@ def run_ours(args):
     if not args.skip_also:
         wl1, _, td1, layer1 = make(ALSO_INDEX)
         ms1, _, _ = device_steps(wl1, td1, layer1, max(3, args.steps // 2), args.warmup, False)
-        also = {"workload": wl1.name, "value": wl1.batch * wl1.img_tokens / (statistics.mean(ms1) / 1e3),
-                "ms_per_step": statistics.mean(ms1)}
+        max1 = dp.max_over_ranks(sum(ms1), world, dev)
+        also = {"workload": wl1.name, "value": dp.aggregate_rate(wl1.batch * wl1.img_tokens, len(ms1), max1, world),
+                "ms_per_step": max1 / len(ms1)}
         layer1.close()
 
     if rank == 0:
@@ -493,7 +477,7 @@ def run_ours(args):
             achieved, peak, unit, bound = by / (avg_top / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
         traffic = kernel_traffic(top)
         cpu = None
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:
             rows = args.cpu_rows
             tcpu = oracle_sample(wl, t_cpu, rows)
             cpu = {"value": wl.batch * rows / tcpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -524,9 +508,7 @@ def run_ours(args):
         }
         print(json.dumps(line), flush=True)
     layer.close()
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    dp.finish(world)
     return 0
 
 

@@ -89,17 +89,26 @@ def _draw(shape, std: float, mean: float, seed: int) -> torch.Tensor:
     return t.to(torch.bfloat16)
 
 
-def make_inputs(wl: Workload, seed_base: int, with_dy: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+# data tensors of data-parallel shard k draw from seed + k * SHARD_STRIDE
+SHARD_STRIDE = 100_000
+_DATA = ("x", "k_cache", "v_cache", "dy")
+
+
+def make_inputs(wl: Workload, seed_base: int, with_dy: Optional[bool] = None,
+                shard: int = 0) -> Dict[str, torch.Tensor]:
     """Return CPU bf16 tensors for one layer call plus ``prefix_len`` (int32).
 
     Shapes: x, dy [B, N, hidden]; w_q [Hq*dh, hidden]; w_k, w_v [Hkv*dh, hidden];
     w_o [hidden, Hq*dh]; q_norm, k_norm [dh]; a_* [r, in]; b_* [out, r];
     k_cache, v_cache [B, Hkv, P, dh] (keys already normalised and rotated).
+    ``shard`` selects a data-parallel shard: the weights are the same for
+    every shard (replicas), x, the cache and dy are drawn independently;
+    shard 0 is the unsharded call.
     """
     d = wl.dims
     B, N, P, r = wl.batch, wl.img_tokens, wl.prefix, wl.lora_rank
     qd, kvd = d.n_q_heads * d.head_dim, d.n_kv_heads * d.head_dim
-    s = lambda name: seed_base + _TENSOR_INDEX[name]
+    s = lambda name: seed_base + _TENSOR_INDEX[name] + (shard * SHARD_STRIDE if name in _DATA else 0)
     out = {
         "x": _draw((B, N, d.hidden), 1.0, 0.0, s("x")),
         "w_q": _draw((qd, d.hidden), 0.02, 0.0, s("w_q")),
@@ -124,8 +133,8 @@ def make_inputs(wl: Workload, seed_base: int, with_dy: Optional[bool] = None) ->
     return out
 
 
-def workload_inputs(index: int, with_dy: Optional[bool] = None) -> Dict[str, torch.Tensor]:
-    return make_inputs(WORKLOADS[index], 1000 * index, with_dy)
+def workload_inputs(index: int, with_dy: Optional[bool] = None, shard: int = 0) -> Dict[str, torch.Tensor]:
+    return make_inputs(WORKLOADS[index], 1000 * index, with_dy, shard)
 
 
 def tiny_workload(batch=2, img_tokens=5, prefix=3, lora_rank=2, lora_alpha=4.0, hidden=64,
