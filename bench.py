@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     "attn_fwd": {"sha256": "fa113b24ee3a31c44f97f0d625781be083da09732a26b1f2e7bfacc173b8f602",
                  "bytes": 104928256 + 32443136},
-    "qkv_gemm": {"sha256": "a3e27cc7e03cf01608307002321cef734c2a77a5a52b7c90a6c75e27712b49b3",
-                 "bytes": 249139456 + 81316096},
+    "qkv_gemm": {"sha256": "de3bed61ebb9ae117c74c0d2d02b7457ea6461a6693ae533928f1bc470c2211f",
+                 "bytes": 275114496 + 81567488},
 }
 KERNEL_SOURCES = {"attn_fwd": "attn_fwd.cuh", "qkv_gemm": "gemm.cuh", "o_gemm": "gemm.cuh"}
 
