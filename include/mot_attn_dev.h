@@ -23,6 +23,19 @@ extern "C" {
 mot_status mot_dev_gemm(const void* a, const void* b, float* d, int32_t m, int32_t n, int32_t k,
                         int32_t is_bf16, int32_t tile_n, void* stream);
 
+/* The other GEMM building blocks on the same operands (A [m, k], B and B2
+ * [n, k], K-major, f16 or bf16; D = f32 [m, n]):
+ *   variant 1: CTA pairs (cluster of 2, cta_group::2), 256 x 256 tiles;
+ *              n a multiple of 256.
+ *   variant 2: 128 x 64 tiles with split-K (f32 partial tiles summed in split
+ *              order by the CTA that completes a tile last); n == 64.
+ *   variant 3: as 2, with B2 as a second B operand of every A tile:
+ *              D = A B^T + A B2^T; n == 64.
+ * k a multiple of 64. Variants 2 and 3 allocate their split scratch and
+ * synchronize `stream` before returning (test entry). */
+mot_status mot_dev_gemm_variant(const void* a, const void* b, const void* b2, float* d, int32_t m, int32_t n,
+                                int32_t k, int32_t is_bf16, int32_t variant, void* stream);
+
 /* Byte offsets, inside the `saved` buffer of a training forward, of the
  * activations it keeps (all device, f16 unless noted):
  *   [0] q^      [B, Hq, N, dh]      normalised + rotated queries

@@ -55,6 +55,8 @@ SIGNATURES = {
     "mot_status_string": (c_char_p, [c_int32]),
     "mot_attn_last_launch_count": (c_int32, [c_void_p]),
     "mot_dev_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p]),
+    "mot_dev_gemm_variant": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int32,
+                                       c_int32, c_void_p]),
     "mot_dev_exp2_poly": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p]),
     "mot_dev_profile": (c_int32, [c_void_p, c_int32]),
     "mot_dev_stage_times": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), c_int32, POINTER(c_int32)]),

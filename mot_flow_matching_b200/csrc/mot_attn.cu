@@ -1289,6 +1289,55 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, in
   return e == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
 }
 
+mot_status mot_dev_gemm_variant(const void* a, const void* b, const void* b2, float* dmat, int32_t m, int32_t n,
+                                int32_t k, int32_t is_bf16, int32_t variant, void* stream) {
+  if (!a || !b || !dmat || m <= 0 || n <= 0 || k <= 0 || variant < 1 || variant > 3) return MOT_ERR_INVALID_ARGUMENT;
+  if (variant == 3 && !b2) return MOT_ERR_INVALID_ARGUMENT;
+  if (k % 64 != 0 || (variant == 1 && n % 256 != 0) || (variant >= 2 && n != 64)) return MOT_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(dmat) || (b2 && !aligned16(b2))) return MOT_ERR_ALIGNMENT;
+  const bool bf = is_bf16 != 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  GemmCore core;
+  EpiStore::Params ep = store_params(m, n);
+  ep.out32 = dmat;
+  ep.ld32 = n;
+  if (variant == 1) {
+    core_init(core, m, n, 256, 128, nullptr);
+    core_pair(core);
+    if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, 128)) return MOT_ERR_CUDA;
+    core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(256, 256, bf, bf), false, false);
+    core.num_segs = 1;
+    return launch_gemm2<256, 6, EpiStore>(core, ep, sms, st) == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+  }
+  // 64-wide tiles with split-K (variant 3: a second B operand on every A tile)
+  core_init(core, m, n, 64, 64, nullptr);
+  if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, 64) ||
+      (variant == 3 && !map2d(&core.maps[3], b2, bf, k, n, k, 64)))
+    return MOT_ERR_CUDA;
+  core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(128, 64, bf, bf), false, false);
+  if (variant == 3) set_dual(core.segs[0], 3);
+  core.num_segs = 1;
+  const int tiles = (m + kBM - 1) / kBM;
+  if (tiles > kSplitCounters) return MOT_ERR_UNSUPPORTED_SHAPE;
+  void* ws = nullptr;
+  int* cnt = nullptr;
+  if (cudaMalloc(&ws, kSplitWsBytes) != cudaSuccess) return MOT_ERR_CUDA;
+  if (cudaMalloc(&cnt, kSplitCounters * sizeof(int)) != cudaSuccess || cudaMemsetAsync(cnt, 0, kSplitCounters * sizeof(int), st) != cudaSuccess) {
+    cudaFree(ws);
+    return MOT_ERR_CUDA;
+  }
+  enable_split(core, ws, cnt);
+  const cudaError_t e = variant == 3 ? launch_gemm_dual<EpiStore>(64, core, ep, sms, st)
+                                     : launch_gemm_narrow<EpiStore>(64, core, ep, sms, st);
+  const cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaFree(ws);
+  cudaFree(cnt);
+  return (e == cudaSuccess && e2 == cudaSuccess) ? MOT_OK : MOT_ERR_CUDA;
+}
+
 mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream) {
   if (!x || !y || n <= 0 || (n & 1)) return MOT_ERR_INVALID_ARGUMENT;
   exp2_poly_kernel<<<(n / 2 + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n / 2);
