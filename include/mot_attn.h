@@ -114,9 +114,10 @@ mot_status mot_attn_query_sizes(const mot_attn_config* cfg, int32_t batch, int32
  * max_img_tokens) and enqueues their initialisation on `stream`. It also
  * allocates the split-K scratch of the LoRA-down GEMMs (f32 partial tiles
  * for up to max_batch * max_img_tokens rows, at most 32 MiB, when
- * lora_rank > 0) with its arrival counters, and, with enable_backward, an
- * f16 copy of w_q|w_k|w_v and a second stream plus two events on which the
- * backward runs the LoRA-gradient GEMMs that feed nothing later in the call.
+ * lora_rank > 0) with its arrival counters, and, with enable_backward,
+ * transposed copies of w_o (bf16) and w_q|w_k|w_v (f16) and a second stream
+ * plus two events on which the backward runs the LoRA-gradient GEMMs that
+ * feed nothing later in the call.
  * Returns MOT_OK and *out, or an error and *out = NULL. */
 mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* weights,
                            void* stream, mot_attn_t* out);

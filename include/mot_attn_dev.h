@@ -31,6 +31,8 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* d, int32_t m, int32
  *              order by the CTA that completes a tile last); n == 64.
  *   variant 3: as 2, with B2 as a second B operand of every A tile:
  *              D = A B^T + A B2^T; n == 64.
+ *   variant 4: as 1, with B given transposed, [k, n] row-major (loaded as an
+ *              MN-major operand): D = A B.
  * k a multiple of 64. Variants 2 and 3 allocate their split scratch and
  * synchronize `stream` before returning (test entry). */
 mot_status mot_dev_gemm_variant(const void* a, const void* b, const void* b2, float* d, int32_t m, int32_t n,

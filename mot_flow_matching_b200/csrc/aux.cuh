@@ -1,6 +1,8 @@
 // aux.cuh -- bandwidth-bound helper kernels (no tensor cores).
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace mot {
@@ -85,6 +87,35 @@ __global__ void __launch_bounds__(256) merge_lora_kernel(const __nv_bfloat16* w,
     for (int k = 0; k < r; ++k) acc = fmaf(sb[threadIdx.y][k], __bfloat162float(a[static_cast<long long>(k) * cols + j]), acc);
     const long long o = static_cast<long long>(i) * cols + j;
     out[o] = __float2bfloat16_rn(fmaf(s, acc, __bfloat162float(w[o])));
+  }
+}
+
+// Transposed copy of a bf16 [rows, cols] matrix into dst [cols, ...] at
+// column offset col_off of rows of length ld_dst: dst[c * ld_dst + col_off + r]
+// = src[r * cols + c], as bf16 or converted to f16 (exact for weights in the
+// f16 range). 32 x 32 tiles through shared memory, reads and writes coalesced.
+template <class OutT>
+__global__ void __launch_bounds__(256) transpose_copy_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
+                                                             OutT* __restrict__ dst, long long ld_dst, int col_off) {
+  __shared__ float tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+#pragma unroll
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < rows && c < cols) ? __bfloat162float(src[static_cast<long long>(r) * cols + c]) : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < cols && r < rows) {
+      const float v = tile[threadIdx.x][i];
+      OutT* o = dst + static_cast<long long>(c) * ld_dst + col_off + r;
+      if constexpr (sizeof(OutT) == 2 && std::is_same<OutT, __half>::value)
+        *o = __float2half_rn(v);
+      else
+        *o = __float2bfloat16_rn(v);
+    }
   }
 }
 

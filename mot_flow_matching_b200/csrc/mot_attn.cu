@@ -365,7 +365,10 @@ struct mot_attn {
   float scale = 0.f;
   int RP = 0;
   __half* wo16 = nullptr;
-  __half* wqkv16 = nullptr;  // [Hq*dh + 2*Hkv*dh, d] f16 copy of W_q|W_k|W_v (backward)
+  // backward: the frozen weights transposed, so that the dO and dx GEMMs read
+  // them as K-major operands
+  __nv_bfloat16* woT = nullptr;  // [Hq*dh, d] bf16, W_o^T
+  __half* wqkvT16 = nullptr;     // [d, Hq*dh + 2*Hkv*dh] f16, [W_q|W_k|W_v]^T
   float* gamma = nullptr;    // [2*dh]: q gain then k gain
   float2* rope = nullptr;
   int rope_len = 0;
@@ -389,7 +392,8 @@ struct mot_attn {
   CUtensorMap wq, wk, wv, wo;  // box rows 128
   CUtensorMap aq, ak, av;      // lora_down q/k/v, box rows RP
   // backward weight maps (MN-major, 64 x 64 boxes)
-  CUtensorMap wo_mn, ao_mn, bo_mn, wq16_mn, wk16_mn, wv16_mn, aq_mn, ak_mn, av_mn;
+  CUtensorMap woT_k, wqkvT_k;  // K-major maps over woT and wqkvT16, box rows 128
+  CUtensorMap ao_mn, bo_mn, aq_mn, ak_mn, av_mn;
 };
 
 namespace {
@@ -406,9 +410,8 @@ mot_status build_weight_maps(mot_attn* h) {
          map2d(&h->av, h->w.a_v, true, d, r, d, box_a);
   }
   if (ok && c.enable_backward) {
-    ok = map2d_mn(&h->wo_mn, h->w.w_o, true, qd, d, qd) && map2d_mn(&h->wq16_mn, h->wqkv16, false, d, qd, d) &&
-         map2d_mn(&h->wk16_mn, h->wqkv16 + qd * d, false, d, kvd, d) &&
-         map2d_mn(&h->wv16_mn, h->wqkv16 + (qd + kvd) * d, false, d, kvd, d);
+    const uint64_t nqkv = qd + 2 * kvd;
+    ok = map2d(&h->woT_k, h->woT, true, d, qd, d, 128) && map2d(&h->wqkvT_k, h->wqkvT16, false, nqkv, d, nqkv, 128);
     if (ok && h->rank > 0) {
       const uint64_t r = h->rank;
       ok = map2d_mn(&h->ao_mn, h->w.a_o, true, qd, r, qd) && map2d_mn(&h->bo_mn, h->w.b_o, true, r, d, r) &&
@@ -419,7 +422,8 @@ mot_status build_weight_maps(mot_attn* h) {
   return ok ? MOT_OK : MOT_ERR_CUDA;
 }
 
-// f16 copies the handle keeps of frozen weights (W_o always; W_q|W_k|W_v for backward)
+// copies the handle keeps of frozen weights: f16 W_o always; for backward
+// W_o^T (bf16) and [W_q|W_k|W_v]^T (f16)
 cudaError_t refresh_f16_copies(mot_attn* h, cudaStream_t s) {
   const mot_attn_config& c = h->cfg;
   const long long d = c.hidden, qd = c.n_q_heads * 128, kvd = c.n_kv_heads * 128;
@@ -428,19 +432,22 @@ cudaError_t refresh_f16_copies(mot_attn* h, cudaStream_t s) {
   jobs.dst[0] = h->wo16;
   jobs.n8[0] = d * qd / 8;
   jobs.count = 1;
+  cvt_multi_kernel<<<4 * h->num_sms, 256, 0, s>>>(jobs, h->status);
   if (c.enable_backward) {
+    const dim3 blk(32, 8);
+    transpose_copy_kernel<__nv_bfloat16><<<dim3((qd + 31) / 32, (d + 31) / 32), blk, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(h->w.w_o), static_cast<int>(d), static_cast<int>(qd), h->woT, d, 0);
     const void* src[3] = {h->w.w_q, h->w.w_k, h->w.w_v};
     const long long rows[3] = {qd, kvd, kvd};
+    const long long nqkv = qd + 2 * kvd;
     long long off = 0;
     for (int i = 0; i < 3; ++i) {
-      jobs.src[1 + i] = static_cast<const __nv_bfloat16*>(src[i]);
-      jobs.dst[1 + i] = h->wqkv16 + off;
-      jobs.n8[1 + i] = rows[i] * d / 8;
-      off += rows[i] * d;
+      transpose_copy_kernel<__half><<<dim3((d + 31) / 32, (rows[i] + 31) / 32), blk, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(src[i]), static_cast<int>(rows[i]), static_cast<int>(d), h->wqkvT16,
+          nqkv, static_cast<int>(off));
+      off += rows[i];
     }
-    jobs.count = 4;
   }
-  cvt_multi_kernel<<<4 * h->num_sms, 256, 0, s>>>(jobs, h->status);
   return cudaGetLastError();
 }
 
@@ -452,7 +459,8 @@ void release(mot_attn* h) {
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->side) cudaStreamDestroy(h->side);
   cudaFree(h->wo16);
-  cudaFree(h->wqkv16);
+  cudaFree(h->wqkvT16);
+  cudaFree(h->woT);
   cudaFree(h->gamma);
   cudaFree(h->rope);
   cudaFree(h->status);
@@ -599,7 +607,8 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
     ok = cudaMalloc(&h->fsplit, h->fsplit_bytes) == cudaSuccess;
   }
   if (ok && cfg->enable_backward)
-    ok = cudaMalloc(&h->wqkv16, (qd + 2 * kvd) * d * 2) == cudaSuccess &&
+    ok = cudaMalloc(&h->wqkvT16, (qd + 2 * kvd) * d * 2) == cudaSuccess &&
+         cudaMalloc(&h->woT, qd * d * 2) == cudaSuccess &&
          cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess &&
          cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
@@ -960,8 +969,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     if (r > 0)
       ok = ok && map2d(&core.maps[1], g_ohi, true, RP, M, RP, 128) && map2d(&core.maps[4], g_olo, true, RP, M, RP, 128);
     if (!ok) return MOT_ERR_CUDA;
-    core.maps[2] = h->wo_mn;
-    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(256, 256, true, true, false, true), false, true);
+    core.maps[2] = h->woT_k;
+    core.segs[0] = seg1(0, 0, 2, d / 64, idesc_f16(256, 256, true, true), false, false);
     core.num_segs = 1;
     if (r > 0) {
       core.maps[3] = h->ao_mn;
@@ -1143,11 +1152,11 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       ok = ok && map2d(&core.maps[1], g_hi, true, 3 * RP, M, 3 * RP, 128) &&
            map2d(&core.maps[8], g_lo, true, 3 * RP, M, 3 * RP, 128);
     if (!ok) return MOT_ERR_CUDA;
-    core.maps[2] = h->wq16_mn;
-    core.maps[3] = h->wk16_mn;
-    core.maps[4] = h->wv16_mn;
-    for (int j = 0; j < 3; ++j)
-      core.segs[j] = seg1(0, col0[j], 2 + j, outj[j] / 64, idesc_f16(256, 256, false, false, false, true), false, true);
+    core.maps[2] = h->wqkvT_k;
+    for (int j = 0; j < 3; ++j) {
+      core.segs[j] = seg1(0, col0[j], 2, outj[j] / 64, idesc_f16(256, 256, false, false), false, false);
+      core.segs[j].b_k0 = col0[j];
+    }
     core.num_segs = 3;
     if (r > 0) {
       core.maps[5] = h->aq_mn;
@@ -1291,9 +1300,10 @@ mot_status mot_dev_gemm(const void* a, const void* b, float* dmat, int32_t m, in
 
 mot_status mot_dev_gemm_variant(const void* a, const void* b, const void* b2, float* dmat, int32_t m, int32_t n,
                                 int32_t k, int32_t is_bf16, int32_t variant, void* stream) {
-  if (!a || !b || !dmat || m <= 0 || n <= 0 || k <= 0 || variant < 1 || variant > 3) return MOT_ERR_INVALID_ARGUMENT;
+  if (!a || !b || !dmat || m <= 0 || n <= 0 || k <= 0 || variant < 1 || variant > 4) return MOT_ERR_INVALID_ARGUMENT;
   if (variant == 3 && !b2) return MOT_ERR_INVALID_ARGUMENT;
-  if (k % 64 != 0 || (variant == 1 && n % 256 != 0) || (variant >= 2 && n != 64)) return MOT_ERR_UNSUPPORTED_SHAPE;
+  if (k % 64 != 0 || ((variant == 1 || variant == 4) && n % 256 != 0) || ((variant == 2 || variant == 3) && n != 64))
+    return MOT_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(a) || !aligned16(b) || !aligned16(dmat) || (b2 && !aligned16(b2))) return MOT_ERR_ALIGNMENT;
   const bool bf = is_bf16 != 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1304,11 +1314,15 @@ mot_status mot_dev_gemm_variant(const void* a, const void* b, const void* b2, fl
   EpiStore::Params ep = store_params(m, n);
   ep.out32 = dmat;
   ep.ld32 = n;
-  if (variant == 1) {
+  if (variant == 1 || variant == 4) {
+    // variant 4: B given as [k, n] (MN-major operand, 64 x 64 boxes)
+    const bool bmn = variant == 4;
     core_init(core, m, n, 256, 128, nullptr);
     core_pair(core);
-    if (!map2d(&core.maps[0], a, bf, k, m, k, 128) || !map2d(&core.maps[2], b, bf, k, n, k, 128)) return MOT_ERR_CUDA;
-    core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(256, 256, bf, bf), false, false);
+    if (!map2d(&core.maps[0], a, bf, k, m, k, 128) ||
+        !(bmn ? map2d_mn(&core.maps[2], b, bf, n, k, n) : map2d(&core.maps[2], b, bf, k, n, k, 128)))
+      return MOT_ERR_CUDA;
+    core.segs[0] = seg1(0, 0, 2, k / 64, idesc_f16(256, 256, bf, bf, false, bmn), false, bmn);
     core.num_segs = 1;
     return launch_gemm2<256, 6, EpiStore>(core, ep, sms, st) == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
   }

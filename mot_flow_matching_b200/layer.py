@@ -115,10 +115,11 @@ def mot_dev_gemm(a, b, d, tile_n=256, stream=None) -> None:
 
 
 def mot_dev_gemm_variant(a, b, d, variant, b2=None, stream=None) -> None:
-    """D = A B^T (+ A B2^T for variant 3) through the pair (1), split-K (2)
-    or dual-B split-K (3) GEMM path; see include/mot_attn_dev.h."""
+    """D = A B^T (+ A B2^T for variant 3; A B with B [k, n] for variant 4)
+    through the pair (1, 4), split-K (2) or dual-B split-K (3) GEMM path;
+    see include/mot_attn_dev.h."""
     m, k = a.shape
-    n = b.shape[0]
+    n = b.shape[1] if variant == 4 else b.shape[0]
     check(lib().mot_dev_gemm_variant(_ptr(a), _ptr(b), _ptr(b2) if b2 is not None else None, _ptr(d), m, n, k,
                                      int(a.dtype == torch.bfloat16), variant, _stream(stream)),
           "mot_dev_gemm_variant")

@@ -84,3 +84,18 @@ def test_dual_b_gemm_matches_float64(cuda_ready, m, k, dtype):
     torch.cuda.synchronize()
     ref = a.double() @ b.double().T + a.double() @ b2.double().T
     assert (d.double() - ref).abs().max().item() <= 4e-5 * k ** 0.5 * ref.abs().max().item()
+
+
+@pytest.mark.parametrize("m,n,k,dtype", [(300, 256, 128, torch.float16), (2048, 1024, 4096, torch.bfloat16)])
+def test_pair_gemm_mn_major_b_matches_float64(cuda_ready, m, n, k, dtype):
+    # CTA pairs with B loaded as an MN-major operand (B given as [k, n])
+    ensure_built()
+    from mot_flow_matching_b200.layer import mot_dev_gemm_variant
+    g = torch.Generator(device="cpu").manual_seed(m + n + k)
+    a = torch.randn(m, k, generator=g).to(dtype).cuda()
+    b = torch.randn(k, n, generator=g).to(dtype).cuda()
+    d = torch.full((m, n), float("nan"), device="cuda")
+    mot_dev_gemm_variant(a, b, d, 4)
+    torch.cuda.synchronize()
+    ref = a.double() @ b.double()
+    assert (d.double() - ref).abs().max().item() <= 2e-5 * k ** 0.5 * ref.abs().max().item()
