@@ -48,7 +48,12 @@ struct GemmSeg {
   // tile is read once for two B operands (a bf16 hi + lo pair)
   int dual;
   int b2_map[kMaxRegions];
+  // 1-CTA kernel: per-region k-block count (0 = kb), for regions that own
+  // fewer K columns than the first
+  int kb_r[kMaxRegions];
 };
+
+__device__ __forceinline__ int seg_kb(const GemmSeg& sg, int reg) { return sg.kb_r[reg] > 0 ? sg.kb_r[reg] : sg.kb; }
 
 struct GemmCore {
   CUtensorMap maps[kMaxMaps];
@@ -61,13 +66,14 @@ struct GemmCore {
   int tiles_m, tiles_n;
   int b_box_rows;  // rows per K-major B TMA box; BN is a multiple of it
   int* status;
-  // split-K (1-CTA kernel only): work item = (tile, split); split s takes
-  // k-blocks [s total_kb / k_splits, (s+1) total_kb / k_splits) of the
-  // concatenated segments and writes its f32 partial tile to split_ws; the
-  // CTA that finishes a tile last (per-tile counter in split_cnt, which it
-  // resets) sums the partials in split order into TMEM and runs the epilogue.
+  // split-K (1-CTA kernel only): work item = (tile, split); split s of a
+  // tile whose segments hold T k-blocks in its region takes k-blocks
+  // [s T / k_splits, (s+1) T / k_splits) of the concatenated segments and
+  // writes its f32 partial tile to split_ws; the CTA that finishes a tile
+  // last (per-tile counter in split_cnt, which it resets) sums the partials
+  // in split order into TMEM and runs the epilogue.
   int k_splits;  // 1 = off
-  int total_kb;
+  int total_kb;  // host side: the smallest K-block total of any tile (bounds the split count)
   float4* split_ws;  // [tiles * k_splits][BN / 4][128]
   int* split_cnt;    // [tiles], zero between launches
   size_t split_cap;  // bytes at split_ws (host side: bounds the split count)
@@ -164,7 +170,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const bool rows_reg = g.regions_on_m != 0;
   const int splits = g.k_splits > 1 ? g.k_splits : 1;
   const int num_items = num_tiles * splits;
-  const int total_kb = g.total_kb;
 
   // Both issuing threads copy what they need out of the parameter block into
   // registers before their K loops: the TMA / MMA wrappers clobber memory, so
@@ -177,15 +182,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int b_box_rows = g.b_box_rows;
       for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
         const int tile = item / splits, split = item - tile * splits;
-        const int kb_lo = split * total_kb / splits, kb_hi = (split + 1) * total_kb / splits;
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
         const int m0 = tm * kBM, n0 = tn * BN;
         const int reg0 = region_of(g, rows_reg ? m0 : n0);
+        int tile_kb = 0;
+        for (int si = 0; si < num_segs; ++si) tile_kb += seg_kb(g.segs[si], reg0);
+        const int kb_lo = split * tile_kb / splits, kb_hi = (split + 1) * tile_kb / splits;
         int gk = 0;  // k-blocks of the segments before this one
         for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
-          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb, a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = seg_kb(sg, reg0), a_k0 = sg.a_k0[reg0], b_k0 = sg.b_k0;
           const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);
           gk += nkb;
           const bool dual = kDual && sg.dual;
@@ -251,8 +258,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
-        const int split = item % splits;
-        const int kb_lo = split * total_kb / splits, kb_hi = (split + 1) * total_kb / splits;
+        const int tile = item / splits, split = item - tile * splits;
+        int tm, tn;
+        tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+        const int reg0 = region_of(g, rows_reg ? tm * kBM : tn * BN);
+        int tile_kb = 0;
+        for (int si = 0; si < num_segs; ++si) tile_kb += seg_kb(g.segs[si], reg0);
+        const int kb_lo = split * tile_kb / splits, kb_hi = (split + 1) * tile_kb / splits;
         mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -260,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         int gk = 0;
         for (int si = 0; si < num_segs; ++si) {
           const GemmSeg& sg = g.segs[si];
-          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = sg.kb;
+          const int a_mn = sg.a_mn, b_mn = sg.b_mn, nkb = seg_kb(sg, reg0);
           const uint32_t idesc = sg.idesc;
           const bool dual = kDual && sg.dual;
           const int kb0 = max(0, kb_lo - gk), kb1 = min(nkb, kb_hi - gk);

@@ -223,8 +223,13 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
   args.core = core;
   args.epi = ep;
   const int tiles = core.tiles_m * core.tiles_n;
-  int total_kb = 0;
-  for (int i = 0; i < core.num_segs; ++i) total_kb += core.segs[i].kb;
+  // every split of every tile needs a k-block: bound by the smallest tile total
+  int total_kb = 1 << 30;
+  for (int r = 0; r < std::max(1, core.num_regions); ++r) {
+    int t = 0;
+    for (int i = 0; i < core.num_segs; ++i) t += core.segs[i].kb_r[r] > 0 ? core.segs[i].kb_r[r] : core.segs[i].kb;
+    total_kb = std::min(total_kb, t);
+  }
   args.core.total_kb = total_kb;
   args.core.k_splits =
       core.k_splits < 0 && tiles <= kSplitCounters ? pick_splits(tiles, total_kb, num_sms, BN, core.split_cap) : 1;
@@ -1075,6 +1080,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       for (int j = 0; j < 3; ++j) {
         core.segs[0].a_k0[j] = col0[j];
         core.segs[0].b_map[j] = 2 + j;
+        core.segs[0].kb_r[j] = outj[j] / 64;  // each block reads only its own K columns
       }
       core.num_segs = 1;
       EpiStore::Params ep = store_params(M, 3 * RP);
