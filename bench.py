@@ -33,6 +33,7 @@ METRIC = "gen-tower attn-layer image tokens/s at 1024²/2048²; % of BF16 tensor
 UNIT = "image tokens/s"
 WORKLOAD_INDEX = 2          # 2048^2 text-to-image CFG layer call
 ALSO_INDEX = 1              # 1024^2 CFG, reported beside it
+EDIT_INDEX = 3              # 2048^2 dual-CFG edit, merged LoRA, reported beside it
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
@@ -457,6 +458,18 @@ def run_ours(args):
         also = {"workload": wl1.name, "value": dp.aggregate_rate(wl1.batch * wl1.img_tokens, len(ms1), max1, world),
                 "ms_per_step": max1 / len(ms1)}
         layer1.close()
+        # the edit workload: adapters baked into the base (merge at load), then rank-0 calls
+        wl3, _, td3, layer3 = make(EDIT_INDEX)
+        merged = {n: torch.empty_like(td3["w_" + n]) for n in ("q", "k", "v", "o")}
+        layer3.merge_lora(merged["q"], merged["k"], merged["v"], merged["o"])
+        ms3, _, _ = device_steps(wl3, td3, layer3, max(3, args.steps // 2), args.warmup, False)
+        max3 = dp.max_over_ranks(sum(ms3), world, dev)
+        fl3 = 4.0 * wl3.batch * wl3.dims.n_q_heads * wl3.img_tokens * (wl3.prefix + wl3.img_tokens) * wl3.dims.head_dim
+        fl3 += 2.0 * wl3.batch * wl3.img_tokens * wl3.dims.hidden * (
+            (wl3.dims.n_q_heads + 2 * wl3.dims.n_kv_heads) * wl3.dims.head_dim + wl3.dims.n_q_heads * wl3.dims.head_dim)
+        also = [also, {"workload": wl3.name, "value": dp.aggregate_rate(wl3.batch * wl3.img_tokens, len(ms3), max3, world),
+                       "ms_per_step": max3 / len(ms3), "tflops": fl3 / (max3 / len(ms3) / 1e3) / 1e12}]
+        layer3.close()
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
