@@ -194,7 +194,9 @@ mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int32_t batch, 
                                     int32_t prefix_max, void* y, float* y_f32, void* stream);
 
 /* Synchronise `stream` and return (and clear) the status latched on the
- * device by earlier calls: MOT_OK, MOT_ERR_NUMERIC or MOT_ERR_TIMEOUT. */
+ * device by earlier calls: MOT_OK, MOT_ERR_NUMERIC or MOT_ERR_TIMEOUT. The
+ * outputs of a call that timed out are undefined; after MOT_ERR_TIMEOUT the
+ * handle's internal split-K counters are reset, so later calls are valid. */
 mot_status mot_attn_get_device_status(mot_attn_t h, void* stream);
 
 /* Free the handle's own device memory. NULL is ignored. */

@@ -654,7 +654,14 @@ mot_status mot_attn_get_device_status(mot_attn_t h, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOT_ERR_CUDA;
   if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOT_ERR_CUDA;
   if (cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) return MOT_ERR_CUDA;
-  if (v & DEV_ERR_TIMEOUT) return MOT_ERR_TIMEOUT;
+  if (v & DEV_ERR_TIMEOUT) {
+    // a GEMM that gave up may have left split-K arrival counters behind:
+    // zero them so that later calls on this handle start clean
+    if (h->side && cudaStreamSynchronize(h->side) != cudaSuccess) return MOT_ERR_CUDA;
+    if (h->split_cnt && cudaMemset(h->split_cnt, 0, 3 * kSplitCounters * sizeof(int)) != cudaSuccess)
+      return MOT_ERR_CUDA;
+    return MOT_ERR_TIMEOUT;
+  }
   if (v & DEV_ERR_NUMERIC) return MOT_ERR_NUMERIC;
   return MOT_OK;
 }
