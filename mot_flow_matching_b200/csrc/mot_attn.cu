@@ -107,7 +107,6 @@ struct Layout {
   // backward scratch (workspace)
   size_t b_do = 0, b_delta = 0, b_dqkv = 0, b_gohi = 0, b_golo = 0, b_go16 = 0, b_ghi = 0, b_glo = 0, b_bqkv16 = 0,
          b_split = 0, bwd_scratch = 0;
-  size_t workspace() const { return std::max(fwd_scratch + act_bytes, bwd_scratch); }
 };
 
 Layout make_layout(const mot_attn_config& c, int B, int N, int P, bool train) {
