@@ -118,3 +118,33 @@ def test_backward_2048sq_train_full(cuda_ready):
     dx, dx32, d_a, d_b, status, _ = run_backward(wl, t)
     assert status == 0
     check_all(wl, t, dx, dx32, d_a, d_b, oracle_backward(wl, t))
+
+
+def test_backward_on_caller_stream(cuda_ready):
+    # forward and backward issued on a caller-created stream: the layer's side
+    # stream work (LoRA gradients) must be joined back into that stream, so
+    # synchronising the caller's stream alone (not the device) is enough to
+    # read every output, and the results equal a default-stream run bit for bit
+    wl = synth.Workload("train_1024sq_b1", 1, 1024, 400, 32, 32.0, train=True)
+    t = synth.make_inputs(wl, 4100, with_dy=True)
+    dx_ref, dx32_ref, da_ref, db_ref, st, layer = run_backward(wl, t)
+    assert st == 0
+    td = to_dev(t)
+    pl = [int(v) for v in t["prefix_len"]]
+    x = td["x"]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        sv = layer.new_saved(*x.shape[:2], td["k_cache"].shape[2])
+        layer.forward(x, td["k_cache"], td["v_cache"], pl, y=torch.empty_like(x), saved=sv, stream=s)
+        dx = torch.empty_like(x)
+        dx32 = torch.empty(x.shape, dtype=torch.float32, device="cuda")
+        d_a = [torch.zeros(td["a_" + n].shape, device="cuda") for n in NAMES]
+        d_b = [torch.zeros(td["b_" + n].shape, device="cuda") for n in NAMES]
+        layer.backward(td["dy"], x, td["k_cache"], td["v_cache"], pl, sv, dx=dx, dx_f32=dx32, d_a=d_a,
+                       d_b=d_b, stream=s)
+        host = [v.cpu() for v in [dx32] + d_a + d_b]  # copies ordered on s only
+    s.synchronize()
+    assert layer.device_status(stream=s) == 0
+    for got, ref in zip(host, [dx32_ref] + da_ref + db_ref):
+        assert torch.equal(got.view(torch.int32), ref.cpu().view(torch.int32))
