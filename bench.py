@@ -268,7 +268,7 @@ def train_steps(bundle, dev, flush, stream, args, world):
     timed separately with CUDA events, per-launch times from the library."""
     import torch
     from mot_flow_matching_b200 import dp
-    from mot_flow_matching_b200.layer import mot_dev_profile, mot_dev_stage_times
+    from mot_flow_matching_b200.layer import mot_dev_profile, mot_dev_stage_timeline, mot_dev_stage_times
     wl, td, layer = bundle
     pl = [int(v) for v in td["prefix_len"]]
     x, kc, vc, dy = td["x"], td["k_cache"], td["v_cache"], td["dy"]
@@ -293,20 +293,29 @@ def train_steps(bundle, dev, flush, stream, args, world):
     for _ in range(args.steps):
         flush.zero_()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        # forward and backward issued back to back, as a training loop does:
+        # nothing on the host waits for the GPU between them
         e[0].record(stream)
         layer.forward(x, kc, vc, pl, y=y, saved=sv, workspace=ws)
         e[1].record(stream)
         launches += layer.last_launch_count()
-        for name, ms in mot_dev_stage_times(layer.handle):
-            stages.setdefault(name, []).append(ms)
         layer.backward(dy, x, kc, vc, pl, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
         e[2].record(stream)
         launches += layer.last_launch_count()
         e[2].synchronize()
         for name, ms in mot_dev_stage_times(layer.handle):
             stages.setdefault(name, []).append(ms)
+        # the backward's launches on one clock (main and side stream), last step
+        timeline = [[n, round(a, 4), round(b, 4)] for n, a, b in mot_dev_stage_timeline(layer.handle)]
         fwd_ms.append(e[0].elapsed_time(e[1]))
         bwd_ms.append(e[1].elapsed_time(e[2]))
+    # per-launch times of the training forward: separate untimed passes (reading
+    # them inside a timed step would stall the host between the two calls)
+    for _ in range(args.steps):
+        flush.zero_()
+        layer.forward(x, kc, vc, pl, y=y, saved=sv, workspace=ws)
+        for name, ms in mot_dev_stage_times(layer.handle):
+            stages.setdefault(name, []).append(ms)
     mot_dev_profile(layer.handle, False)
     assert layer.device_status() == 0
     layer.close()
@@ -325,7 +334,8 @@ def train_steps(bundle, dev, flush, stream, args, world):
     return {"workload": wl.name, "fwd_ms": f, "bwd_ms": b, "tokens_per_s": world * wl.batch * wl.img_tokens / ((f + b) / 1e3),
             "fwd_tflops": fwd_flops / (f / 1e3) / 1e12, "bwd_tflops": bwd_flops / (b / 1e3) / 1e12,
             "bwd_pct_of_bf16_peak": 100.0 * bwd_flops / (b / 1e3) / 1e12 / peaks["bf16_tflops"],
-            "bwd_algorithmic_gflop": bwd_flops / 1e9, "gpu_launches": launches * world, "stages": per}
+            "bwd_algorithmic_gflop": bwd_flops / 1e9, "gpu_launches": launches * world, "stages": per,
+            "bwd_timeline_ms": timeline}
 
 
 def run_ours(args):

@@ -62,6 +62,15 @@ mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32
 mot_status mot_dev_profile(mot_attn_t h, int32_t enable);
 mot_status mot_dev_stage_times(mot_attn_t h, int32_t* ids, float* ms, int32_t max, int32_t* count);
 
+/* The same launches placed on one clock: t0_ms[i] / t1_ms[i] are the times
+ * of launch i's start and end events, in milliseconds after the first
+ * launch's start event. Side-stream launches (the backward's LoRA gradients)
+ * start at the side stream's own previous event, so overlap between the two
+ * streams shows as intersecting intervals. Same argument rules as
+ * mot_dev_stage_times. */
+mot_status mot_dev_stage_timeline(mot_attn_t h, int32_t* ids, float* t0_ms, float* t1_ms, int32_t max,
+                                  int32_t* count);
+
 /* y[i] = 2^x[i] through the FMA-pipe exponential the attention softmax uses
  * for part of its probabilities (range reduction + degree-3 polynomial);
  * x, y device f32 [n], n even, x in [-125, 8]. For accuracy tests. */

@@ -678,6 +678,39 @@ struct EpiStore {
       }
     }
   }
+  // bf16 or f16 pair (a in the low half), round to nearest even
+  template <bool kBf16>
+  __device__ __forceinline__ static uint32_t pack2(float a, float b) {
+    if constexpr (kBf16) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+      return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+      const __half2 h = __floats2half2_rn(a, b);
+      return *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  // 32 full columns of one output, its type and kind fixed at compile time:
+  // straight-line packed conversions and four 16-byte stores. kResid: the
+  // bf16 residual of a bf16 output scaled by `scale`. f16: amax collects the
+  // largest magnitude (NaN propagates) for the overflow check.
+  template <bool kBf16, bool kResid>
+  __device__ __forceinline__ static void store32(uint16_t* row, const float (&v)[32], float scale, float& amax) {
+    uint32_t w[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float a = v[2 * k] * scale, b = v[2 * k + 1] * scale;
+      if constexpr (kResid) {
+        const uint32_t hi = pack2<true>(a, b);
+        a -= __uint_as_float(hi << 16);
+        b -= __uint_as_float(hi & 0xffff0000u);
+      }
+      if constexpr (!kBf16) amax = fmax3_nan(amax, fabsf(a), fabsf(b));
+      w[k] = pack2<kBf16>(a, b);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(row);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
   template <int BN>
   __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
                                                int* status) {
@@ -685,42 +718,72 @@ struct EpiStore {
     bool overflow = false;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
+      const int n = n0 + c;
+      if (n >= p.N) break;  // the same for every thread: no TMEM load for columns past N
       float v[32];
       load_row32(taddr + c, v);
-      const int n = n0 + c;
-      if (m >= p.M || n >= p.N) continue;
+      if (m >= p.M) continue;
       const int ncols = min(32, p.N - n);
 #pragma unroll 1
-      for (int i = 0; i < 3; ++i)
-        if (p.o16[i].ptr) store16(p, i, m, n, v, ncols, overflow);
-      if (p.out32) {
-        // every old value is loaded before the first store, so the loads
-        // overlap instead of each waiting for the store before it
-        if (p.transpose32) {
-          float old[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            old[k] = (p.accumulate32 && k < ncols) ? p.out32[static_cast<long long>(n + k) * p.ld32 + m] : 0.f;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (k < ncols) p.out32[static_cast<long long>(n + k) * p.ld32 + m] = fmaf(v[k], p.scale32, old[k]);
-        } else if (ncols == 32) {
-          float4* dst = reinterpret_cast<float4*>(p.out32 + m * p.ld32 + n);
-          float4 old[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) old[i] = p.accumulate32 ? dst[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(fmaf(v[4 * i], p.scale32, old[i].x), fmaf(v[4 * i + 1], p.scale32, old[i].y),
-                                 fmaf(v[4 * i + 2], p.scale32, old[i].z), fmaf(v[4 * i + 3], p.scale32, old[i].w));
+      for (int i = 0; i < 3; ++i) {
+        const Out16& o = p.o16[i];
+        if (!o.ptr) continue;
+        uint16_t* row16 = static_cast<uint16_t*>(o.ptr) + static_cast<long long>(m) * o.ld + n;
+        const bool aligned = (reinterpret_cast<uintptr_t>(row16) & 15) == 0;
+        const bool resid = o.residual_of >= 0;
+        const Out16& hi = p.o16[resid ? o.residual_of : i];
+        if (ncols == 32 && aligned && (!resid || (hi.bf16 && o.bf16))) {
+          float amax = 0.f;
+          if (resid)
+            store32<true, true>(row16, v, hi.scale, amax);
+          else if (o.bf16)
+            store32<true, false>(row16, v, o.scale, amax);
+          else
+            store32<false, false>(row16, v, o.scale, amax);
+          overflow |= p.check_f16 && !o.bf16 && !(amax <= 65504.f);
         } else {
-          float* o = p.out32 + m * p.ld32 + n;
+          store16(p, i, m, n, v, ncols, overflow);
+        }
+      }
+      if (p.out32) {
+        const float s32 = p.scale32;
+        if (p.transpose32) {
+          // element (m, n + k) at out32[(n + k) ld32 + m]: for each k a warp
+          // writes 32 consecutive floats; old values first, then the stores
+          const long long ld = p.ld32;
+          float* base = p.out32 + static_cast<long long>(n) * ld + m;
           float old[32];
+          if (ncols == 32) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) old[k] = (p.accumulate32 && k < ncols) ? o[k] : 0.f;
+            for (int k = 0; k < 32; ++k) old[k] = p.accumulate32 ? base[k * ld] : 0.f;
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (k < ncols) o[k] = fmaf(v[k], p.scale32, old[k]);
+            for (int k = 0; k < 32; ++k) base[k * ld] = fmaf(v[k], s32, old[k]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) old[k] = (p.accumulate32 && k < ncols) ? base[k * ld] : 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < ncols) base[k * ld] = fmaf(v[k], s32, old[k]);
+          }
+        } else {
+          float* o = p.out32 + static_cast<long long>(m) * p.ld32 + n;
+          if (ncols == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+            float4* dst = reinterpret_cast<float4*>(o);
+            float4 old[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) old[q] = p.accumulate32 ? dst[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(fmaf(v[4 * q], s32, old[q].x), fmaf(v[4 * q + 1], s32, old[q].y),
+                                   fmaf(v[4 * q + 2], s32, old[q].z), fmaf(v[4 * q + 3], s32, old[q].w));
+          } else {
+            float old[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) old[k] = (p.accumulate32 && k < ncols) ? o[k] : 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k < ncols) o[k] = fmaf(v[k], s32, old[k]);
+          }
         }
       }
     }
@@ -736,7 +799,7 @@ struct EpiLoraGrad {
   struct Params {
     float* out[3];
     long long ld;
-    int RP, r, M;
+    int RP, r, M;  // RP: a multiple of 32, so a 32-column chunk lies in one block
     int transpose, accumulate;
   };
   template <int BN>
@@ -745,24 +808,52 @@ struct EpiLoraGrad {
     const int m = m0 + row;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
+      // block j and its first column k0: the same for every thread, so chunks
+      // of padding columns (k0 >= r) or past the three blocks skip the TMEM load
+      const int n = n0 + c;
+      const int j = n / p.RP, k0 = n - j * p.RP;
+      const int nv = j > 2 ? 0 : min(32, p.r - k0);
+      if (nv <= 0) continue;
       float v[32];
       load_row32(taddr + c, v);
       if (m >= p.M) continue;
-      // old values first (independent loads), then the stores
-      float* dst[32];
+      float* out = j == 0 ? p.out[0] : j == 1 ? p.out[1] : p.out[2];
       float old[32];
+      if (p.transpose) {
+        // element (m, k) at out[k ld + m]: a warp's 32 rows are 32 consecutive floats
+        const long long ld = p.ld;
+        float* base = out + static_cast<long long>(k0) * ld + m;
+        if (nv == 32) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int n = n0 + c + i;
-        const int j = n / p.RP, k = n - j * p.RP;
-        dst[i] = (j > 2 || k >= p.r) ? nullptr
-                 : p.transpose       ? p.out[j] + static_cast<long long>(k) * p.ld + m
-                                     : p.out[j] + m * p.ld + k;
-        old[i] = (p.accumulate && dst[i]) ? *dst[i] : 0.f;
+          for (int i = 0; i < 32; ++i) old[i] = p.accumulate ? base[i * ld] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) base[i * ld] = old[i] + v[i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) old[i] = (p.accumulate && i < nv) ? base[i * ld] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) base[i * ld] = old[i] + v[i];
+        }
+      } else {
+        float* base = out + static_cast<long long>(m) * p.ld + k0;
+        if (nv == 32 && (reinterpret_cast<uintptr_t>(base) & 15) == 0) {
+          float4* dst = reinterpret_cast<float4*>(base);
+          float4 o4[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) o4[q] = p.accumulate ? dst[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(o4[q].x + v[4 * q], o4[q].y + v[4 * q + 1], o4[q].z + v[4 * q + 2],
+                                 o4[q].w + v[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) old[i] = (p.accumulate && i < nv) ? base[i] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) base[i] = old[i] + v[i];
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (dst[i]) *dst[i] = old[i] + v[i];
     }
   }
 };
@@ -785,16 +876,31 @@ struct EpiRowBlocks {
     const int j = (m >= p.row0[1]) + (m >= p.row0[2]);
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
+      const int n = n0 + c;
+      if (n >= p.cols) break;  // the same for every thread: no TMEM load for padding columns
       float v[32];
       load_row32(taddr + c, v);
       if (m >= p.row0[3]) continue;
-      float* o = p.out[j] + static_cast<long long>(m - p.row0[j]) * p.ld;
-      float old[32];
+      const int nv = min(32, p.cols - n);
+      float* o = (j == 0 ? p.out[0] : j == 1 ? p.out[1] : p.out[2]) +
+                 static_cast<long long>(m - p.row0[j]) * p.ld + n;
+      if (nv == 32 && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+        float4* dst = reinterpret_cast<float4*>(o);
+        float4 o4[8];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) old[i] = (p.accumulate && n0 + c + i < p.cols) ? o[n0 + c + i] : 0.f;
+        for (int q = 0; q < 8; ++q) o4[q] = p.accumulate ? dst[q] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (n0 + c + i < p.cols) o[n0 + c + i] = old[i] + v[i];
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(o4[q].x + v[4 * q], o4[q].y + v[4 * q + 1], o4[q].z + v[4 * q + 2],
+                               o4[q].w + v[4 * q + 3]);
+      } else {
+        float old[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) old[i] = (p.accumulate && i < nv) ? o[i] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < nv) o[i] = old[i] + v[i];
+      }
     }
   }
 };

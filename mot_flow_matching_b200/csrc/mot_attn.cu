@@ -1395,6 +1395,24 @@ mot_status mot_dev_stage_times(mot_attn_t h, int32_t* ids, float* ms, int32_t ma
   return MOT_OK;
 }
 
+mot_status mot_dev_stage_timeline(mot_attn_t h, int32_t* ids, float* t0_ms, float* t1_ms, int32_t max,
+                                  int32_t* count) {
+  if (!h || !ids || !t0_ms || !t1_ms || max < 0 || !count) return MOT_ERR_INVALID_ARGUMENT;
+  if (!h->profile) return MOT_ERR_INVALID_ARGUMENT;
+  *count = h->stage_count;
+  if (h->stage_count == 0) return MOT_OK;
+  cudaEvent_t origin = h->stage_start[0];
+  for (int i = 0; i < h->stage_count && i < max; ++i) {
+    ids[i] = h->stage_ids[i];
+    if (!origin || !h->stage_start[i] || !h->stage_end[i]) return MOT_ERR_CUDA;
+    if (cudaEventSynchronize(h->stage_end[i]) != cudaSuccess ||
+        cudaEventElapsedTime(&t0_ms[i], origin, h->stage_start[i]) != cudaSuccess ||
+        cudaEventElapsedTime(&t1_ms[i], origin, h->stage_end[i]) != cudaSuccess)
+      return MOT_ERR_CUDA;
+  }
+  return MOT_OK;
+}
+
 const char* mot_dev_stage_name(int32_t id) {
   if (id >= 0 && id < static_cast<int32_t>(sizeof(kStageNames) / sizeof(kStageNames[0]))) return kStageNames[id];
   return "?";

@@ -149,6 +149,17 @@ def mot_dev_stage_times(h, max_stages: int = 32):
     return [(lib().mot_dev_stage_name(ids[i]).decode(), ms[i]) for i in range(min(count.value, max_stages))]
 
 
+def mot_dev_stage_timeline(h, max_stages: int = 32):
+    """[(stage name, start ms, end ms)] of the last call's launches on one clock
+    (milliseconds after the first launch's start)."""
+    ids = (c_int32 * max_stages)()
+    t0 = (ctypes.c_float * max_stages)()
+    t1 = (ctypes.c_float * max_stages)()
+    count = c_int32(0)
+    check(lib().mot_dev_stage_timeline(h, ids, t0, t1, max_stages, byref(count)), "mot_dev_stage_timeline")
+    return [(lib().mot_dev_stage_name(ids[i]).decode(), t0[i], t1[i]) for i in range(min(count.value, max_stages))]
+
+
 class MotAttnLayer:
     """A handle plus the caller-owned buffers of one call shape."""
 
