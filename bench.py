@@ -288,7 +288,6 @@ def train_steps(bundle, dev, flush, stream, args, world):
         step()
     torch.cuda.synchronize(dev)
     dp.barrier(world)
-    mot_dev_profile(layer.handle, True)
     fwd_ms, bwd_ms, stages, launches = [], [], {}, 0
     for _ in range(args.steps):
         flush.zero_()
@@ -303,19 +302,22 @@ def train_steps(bundle, dev, flush, stream, args, world):
         e[2].record(stream)
         launches += layer.last_launch_count()
         e[2].synchronize()
-        for name, ms in mot_dev_stage_times(layer.handle):
-            stages.setdefault(name, []).append(ms)
-        # the backward's launches on one clock (main and side stream), last step
-        timeline = [[n, round(a, 4), round(b, 4)] for n, a, b in mot_dev_stage_timeline(layer.handle)]
         fwd_ms.append(e[0].elapsed_time(e[1]))
         bwd_ms.append(e[1].elapsed_time(e[2]))
-    # per-launch times of the training forward: separate untimed passes (reading
-    # them inside a timed step would stall the host between the two calls)
+    # per-launch times from separate untimed passes (the profiling events sit
+    # between launches; reading them inside a timed step would also stall the
+    # host between the two calls)
+    mot_dev_profile(layer.handle, True)
     for _ in range(args.steps):
         flush.zero_()
         layer.forward(x, kc, vc, pl, y=y, saved=sv, workspace=ws)
         for name, ms in mot_dev_stage_times(layer.handle):
             stages.setdefault(name, []).append(ms)
+        layer.backward(dy, x, kc, vc, pl, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
+        for name, ms in mot_dev_stage_times(layer.handle):
+            stages.setdefault(name, []).append(ms)
+        # the backward's launches on one clock (main and side stream), last pass
+        timeline = [[n, round(a, 4), round(b, 4)] for n, a, b in mot_dev_stage_timeline(layer.handle)]
     mot_dev_profile(layer.handle, False)
     assert layer.device_status() == 0
     layer.close()
@@ -385,7 +387,6 @@ def run_ours(args):
         for _ in range(warmup):
             layer.forward(x, kc, vc, pl, y=y, workspace=ws)
         torch.cuda.synchronize(dev)
-        mot_dev_profile(layer.handle, profile)
         dp.barrier(world)
         torch.cuda.synchronize(dev)
         step_ms, stages = [], {}
@@ -400,11 +401,19 @@ def run_ours(args):
             launches += layer.last_launch_count()
             e1.synchronize()
             step_ms.append(e0.elapsed_time(e1))
-            if profile:
+        torch.cuda.synchronize(dev)
+        if profile:
+            # per-launch times from separate passes: the library's profiling
+            # events sit between launches and would keep consecutive kernels
+            # from overlapping their prologues (programmatic launch)
+            mot_dev_profile(layer.handle, True)
+            for _ in range(steps):
+                flush.zero_()
+                layer.forward(x, kc, vc, pl, y=y, workspace=ws)
                 for name, ms in mot_dev_stage_times(layer.handle):
                     stages.setdefault(name, []).append(ms)
-        torch.cuda.synchronize(dev)
-        mot_dev_profile(layer.handle, False)
+            mot_dev_profile(layer.handle, False)
+            torch.cuda.synchronize(dev)
         return step_ms, stages, launches
 
     wl, t_cpu, td, layer = make(WORKLOAD_INDEX)

@@ -678,6 +678,8 @@ __global__ void __launch_bounds__(kAttnBwdThreads, 1) attn_bwd_kernel(const __gr
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int bid = static_cast<int>(blockIdx.x);
+  grid_dep_launch();
+  grid_dep_wait();
   if (bid < p.dkv_ctas)
     attn_bwd_dkv_cta(p, bid, smem);
   else

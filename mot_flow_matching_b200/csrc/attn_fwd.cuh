@@ -148,8 +148,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   const int h = bid % p.Hq;
   const int b = bid / p.Hq;
   const int g = h / (p.Hq / p.Hkv);
-  const int L = p.plen[b] + p.N;
-  const int T = (L + 127) >> 7;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -173,6 +171,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();
+  grid_dep_wait();  // inputs of this call (q^, K, V, prefix lengths) are final from here on
+  const int L = p.plen[b] + p.N;
+  const int T = (L + 127) >> 7;
   const WaitGuard wg{abort_flag, p.status};
 
   if (warp == 0) {

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(256) build_kv_kernel(const __nv_bfloat16* __re
                                                        __half* __restrict__ kall, __half* __restrict__ vall,
                                                        int Hkv, int Pmax, int N, int Lcap, long long total_chunks,
                                                        PlenArray plen, int* status) {
+  grid_dep_launch();
+  grid_dep_wait();
   bool overflow = false;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total_chunks;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -129,6 +131,8 @@ struct CvtJobs {
 };
 
 __global__ void __launch_bounds__(256) cvt_multi_kernel(const CvtJobs jobs, int* status) {
+  grid_dep_launch();
+  grid_dep_wait();
   bool overflow = false;
   for (int j = 0; j < jobs.count; ++j) {
     const uint4* src = reinterpret_cast<const uint4*>(jobs.src[j]);

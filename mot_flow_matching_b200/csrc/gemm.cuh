@@ -165,6 +165,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitGuard wg{abort_flag, g.status};
+  grid_dep_launch();
+  grid_dep_wait();  // every global access of this kernel comes after this
 
   const int num_tiles = g.tiles_m * g.tiles_n;
   const bool rows_reg = g.regions_on_m != 0;
@@ -472,6 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitGuard wg{abort_flag, g.status};
+  grid_dep_launch();
+  grid_dep_wait();  // every global access of this kernel comes after this
 
   const int num_tiles = g.tiles_m * g.tiles_n;  // 256-row tiles
   const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;

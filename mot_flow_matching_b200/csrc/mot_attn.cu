@@ -202,6 +202,27 @@ void set_dual(GemmSeg& sg, int b2) {
   for (int i = 0; i < kMaxRegions; ++i) sg.b2_map[i] = b2;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream drains (once all that kernel's CTAs
+// are running) and runs its prologue (barriers, TMEM, descriptor prefetch);
+// its grid_dep_wait then holds every global access until the previous grid
+// has completed. Every kernel launched this way calls grid_dep_wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const Args&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // let launch_gemm split K (1-CTA kernel; partials in ws of cap bytes, counters in cnt)
 void enable_split(GemmCore& c, void* ws, int* cnt, size_t cap = kSplitWsBytes) {
   c.k_splits = -1;
@@ -234,8 +255,7 @@ cudaError_t launch_gemm(const GemmCore& core, const typename Epi::Params& ep, in
       core.k_splits < 0 && tiles <= kSplitCounters ? pick_splits(tiles, total_kb, num_sms, BN, core.split_cap) : 1;
   const int items = tiles * args.core.k_splits;
   const int grid = std::max(1, std::min(items, num_sms));
-  kern<<<grid, kGemmThreads, L::kBytes, st>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kGemmThreads), L::kBytes, st, args);
 }
 
 // CTA pairs a pair-kernel launch of `tiles` tiles uses: the fewest that
@@ -264,8 +284,7 @@ cudaError_t launch_gemm2(const GemmCore& core, const typename Epi::Params& ep, i
   // pair gets the same tile count, and the SMs left over can run other work
   // (the backward's side-stream GEMMs) for the whole duration
   const int pairs = pair_count(core.tiles_m * core.tiles_n, num_sms);
-  kern<<<2 * pairs, kGemmThreads, L::kBytes, st>>>(args);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kGemmThreads), L::kBytes, st, args);
 }
 
 // tiles of the pair kernel: 256 rows of D per CTA pair
@@ -724,8 +743,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
       jobs.n8[i] = n[i] / 8;
     }
     jobs.count = 5;
-    cvt_multi_kernel<<<2 * h->num_sms, 256, 0, st>>>(jobs, h->status);
-    lz.done(cudaGetLastError());
+    lz.done(launch_pdl(cvt_multi_kernel, dim3(2 * h->num_sms), dim3(256), 0, st, jobs, h->status));
   }
   // 2. key/value buffers: prefix rows + zero tail
   lz.stage = ST_BUILD_KV;
@@ -734,10 +752,9 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     for (int b = 0; b < B; ++b) pl.v[b] = prefix_len[b];
     const long long chunks = static_cast<long long>(B) * Hkv * L.Lcap * 16;
     const int grid = static_cast<int>(std::min<long long>((chunks + 255) / 256, 16LL * h->num_sms));
-    build_kv_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_cache),
-                                          static_cast<const __nv_bfloat16*>(v_cache), k_all, v_all, Hkv,
-                                          std::max(P, 1), N, L.Lcap, chunks, pl, h->status);
-    lz.done(cudaGetLastError());
+    lz.done(launch_pdl(build_kv_kernel, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(k_cache),
+                       static_cast<const __nv_bfloat16*>(v_cache), k_all, v_all, Hkv, std::max(P, 1), N, L.Lcap,
+                       chunks, pl, h->status));
   }
   // 3. LoRA down for q/k/v: u_qkv[:, j*RP:(j+1)*RP] = s x A_j^T (f16)
   lz.stage = ST_LORA_DOWN_QKV;
@@ -832,8 +849,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ap.status = h->status;
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(attn_fwd_kernel, AttnSmem::kBytes); });
-    attn_fwd_kernel<<<B * Hq * ap.q_pairs, kAttnThreads, AttnSmem::kBytes, st>>>(ap);
-    lz.done(cudaGetLastError());
+    lz.done(launch_pdl(attn_fwd_kernel, dim3(B * Hq * ap.q_pairs), dim3(kAttnThreads), AttnSmem::kBytes, st, ap));
   }
   // 6. LoRA down for o: u_o = s o A_o^T (f16; training also keeps it as a bf16 hi + lo pair)
   lz.stage = ST_LORA_DOWN_O;
@@ -952,8 +968,7 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
       jobs.n8[j] = static_cast<long long>(outj[j]) * r / 8;
     }
     jobs.count = 3;
-    cvt_multi_kernel<<<64, 256, 0, st>>>(jobs, h->status);
-    lz.done(cudaGetLastError());
+    lz.done(launch_pdl(cvt_multi_kernel, dim3(64), dim3(256), 0, st, jobs, h->status));
     // g_o = dy B_o  -> s g_o as bf16 hi + lo, and as f16
     lz.stage = ST_BWD_G_O;
     GemmCore core;
@@ -1065,8 +1080,8 @@ mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(attn_bwd_kernel, AttnBwdSmem::kBytes); });
     lz.stage = ST_BWD_ATTN;
-    attn_bwd_kernel<<<ap.dkv_ctas + B * Hq * ap.q_tiles, kAttnBwdThreads, AttnBwdSmem::kBytes, st>>>(ap);
-    lz.done(cudaGetLastError());
+    lz.done(launch_pdl(attn_bwd_kernel, dim3(ap.dkv_ctas + B * Hq * ap.q_tiles), dim3(kAttnBwdThreads),
+                       AttnBwdSmem::kBytes, st, ap));
   }
   if (r > 0) {
     {

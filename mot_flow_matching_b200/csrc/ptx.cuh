@@ -400,6 +400,16 @@ __device__ __forceinline__ uint32_t pack_bf162(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Programmatic dependent launch. grid_dep_wait: block until every grid this
+// one depends on in its stream has completed and its memory is visible (a
+// no-op when the launch did not allow programmatic serialization); nothing
+// before it may touch global memory that earlier kernels write or read.
+// grid_dep_launch: let the next kernel of the stream launch once every CTA of
+// this grid has issued it (or exited), so its prologue overlaps this grid's
+// tail; the next kernel still waits in its own grid_dep_wait.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
