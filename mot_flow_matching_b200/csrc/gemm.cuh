@@ -92,9 +92,11 @@ __device__ __forceinline__ int region_of(const GemmCore& g, int n) {
   return i;
 }
 
-// grouped tile order: 8 M-tiles share each sweep over N (L2 reuse of A rows)
+// grouped tile order: 16 M-tiles share each sweep over N, so A's rows stay in
+// L2 across the sweep and B is streamed once per group (the 8192-row QKV
+// projection reads its 50 MB of weights twice instead of four times)
 __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& tm, int& tn) {
-  constexpr int G = 8;
+  constexpr int G = 16;
   const int per_group = G * tiles_n;
   const int group = tile / per_group;
   const int first_m = group * G;
