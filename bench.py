@@ -40,10 +40,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the 2048^2 CFG workload, keyed by the sha256 of the
 # kernel's source file at capture time: a changed kernel reports null.
 TRAFFIC = {
-    "attn_fwd": {"sha256": "fa113b24ee3a31c44f97f0d625781be083da09732a26b1f2e7bfacc173b8f602",
-                 "bytes": 104928256 + 32443136},
-    "qkv_gemm": {"sha256": "de3bed61ebb9ae117c74c0d2d02b7457ea6461a6693ae533928f1bc470c2211f",
-                 "bytes": 275114496 + 81567488},
+    "attn_fwd": {"sha256": "bdc599b623238d957f063bc5acac4a7266ff1705f724d6ff19c0fb05ebd75e5d",
+                 "bytes": 104960512 + 33044224},
+    "qkv_gemm": {"sha256": "9cc99ea8dda5aee19ed56221282f43d36bd6c96740405226bbd7867286c344cf",
+                 "bytes": 221264128 + 81383936},
 }
 KERNEL_SOURCES = {"attn_fwd": "attn_fwd.cuh", "qkv_gemm": "gemm.cuh", "o_gemm": "gemm.cuh"}
 
