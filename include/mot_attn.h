@@ -193,6 +193,42 @@ mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int32_t batch, 
                                     const void* k_cache, const void* v_cache, const int32_t* prefix_len,
                                     int32_t prefix_max, void* y, float* y_f32, void* stream);
 
+/* Device staging bytes mot_attn_forward_host needs for calls of this shape:
+ * two slots, each holding one call's x, k_cache, v_cache and y. Host-only;
+ * no CUDA calls. */
+mot_status mot_attn_query_host_staging(const mot_attn_config* cfg, int32_t batch, int32_t img_tokens,
+                                       int32_t prefix_max, size_t* staging_bytes);
+
+/* `steps` inference forwards whose inputs and outputs live in host memory
+ * (the pages describe no such call: it is the host-buffer path a serving
+ * loop or an end-to-end measurement drives).
+ *   x_host[i]        host bf16 [B, N, d]              input of call i
+ *   k_cache_host[i], v_cache_host[i]
+ *                    host bf16 [B, Hkv, P_max, dh]     (NULL allowed when P_max == 0)
+ *   prefix_len       host int32 [B], shared by all calls
+ *   y_host[i]        host bf16 [B, N, d]              output of call i
+ *   staging          device, staging_bytes from mot_attn_query_host_staging
+ *   workspace        device, workspace_bytes from mot_attn_query_sizes
+ * Call i uses staging slot i % 2: its inputs are copied into the slot on a
+ * copy-in stream the handle owns, the layer runs on `stream` (as
+ * mot_attn_forward), and y is copied back on a copy-out stream the handle
+ * owns; the copy-in of call i+1 and the copy-out of call i-1 therefore
+ * overlap the layer of call i (PCIe carries both directions at once). A slot
+ * is refilled only after the layer two calls earlier has read it and its y
+ * has been copied out. Exception to the host-pointer rule above: the host
+ * buffers are read and written asynchronously, after this function returns;
+ * they must stay valid and untouched until `stream` has completed the work
+ * enqueued so far. Page-locked (pinned) host memory lets the copies overlap;
+ * pageable memory gives the same results with the copies serialised.
+ * Both copy streams first wait for the work already enqueued on `stream`,
+ * and `stream` finally waits for the last copy-out, so every y_host[i] is
+ * complete once `stream` reaches the end of this call's work. */
+mot_status mot_attn_forward_host(mot_attn_t h, int32_t steps, const void* const* x_host, int32_t batch,
+                                 int32_t img_tokens, const void* const* k_cache_host,
+                                 const void* const* v_cache_host, const int32_t* prefix_len, int32_t prefix_max,
+                                 void* const* y_host, void* staging, size_t staging_bytes, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream` and return (and clear) the status latched on the
  * device by earlier calls: MOT_OK, MOT_ERR_NUMERIC or MOT_ERR_TIMEOUT. The
  * outputs of a call that timed out are undefined; after MOT_ERR_TIMEOUT the

@@ -49,6 +49,11 @@ SIGNATURES = {
                                     POINTER(c_void_p), POINTER(c_void_p), c_int32, c_void_p, c_size_t, c_void_p]),
     "mot_attn_forward_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                            POINTER(c_int32), c_int32, c_void_p, c_void_p, c_void_p]),
+    "mot_attn_query_host_staging": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32,
+                                              POINTER(c_size_t)]),
+    "mot_attn_forward_host": (c_int32, [c_void_p, c_int32, POINTER(c_void_p), c_int32, c_int32, POINTER(c_void_p),
+                                        POINTER(c_void_p), POINTER(c_int32), c_int32, POINTER(c_void_p), c_void_p,
+                                        c_size_t, c_void_p, c_size_t, c_void_p]),
     "mot_attn_merge_lora": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "mot_attn_get_device_status": (c_int32, [c_void_p, c_void_p]),
     "mot_attn_destroy": (None, [c_void_p]),

@@ -92,6 +92,19 @@ bool map3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// one staging slot of the host-buffer forward: x, y, k_cache, v_cache, each
+// 256-byte aligned
+struct HostStaging {
+  size_t x, kv, slot;
+};
+HostStaging host_staging(const mot_attn_config& c, int B, int N, int P) {
+  HostStaging s;
+  s.x = round_up(static_cast<size_t>(B) * N * c.hidden * 2, 256);
+  s.kv = round_up(static_cast<size_t>(B) * c.n_kv_heads * P * c.head_dim * 2, 256);
+  s.slot = 2 * s.x + 2 * s.kv;
+  return s;
+}
+
 // ------------------------------------------------------------------ layouts
 // split-K partial tiles of the LoRA-gradient GEMMs (backward workspace)
 constexpr size_t kSplitWsBytes = size_t(16) << 20;
@@ -404,6 +417,10 @@ struct mot_attn {
   // backward: a second stream for the gradient GEMMs nothing later depends on
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  // host-buffer forward: copy-in and copy-out streams and per-slot events,
+  // made on first use
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t hev_start = nullptr, hev_in[2] = {}, hev_comp[2] = {}, hev_out[2] = {};
   // optional per-launch timing (mot_dev_profile): a start and an end event
   // per launch, on the stream it ran on
   bool profile = false;
@@ -481,6 +498,12 @@ void release(mot_attn* h) {
   if (h->ev_fork) cudaEventDestroy(h->ev_fork);
   if (h->ev_join) cudaEventDestroy(h->ev_join);
   if (h->side) cudaStreamDestroy(h->side);
+  const cudaEvent_t hev[] = {h->hev_start, h->hev_in[0], h->hev_in[1], h->hev_comp[0], h->hev_comp[1],
+                             h->hev_out[0], h->hev_out[1]};
+  for (cudaEvent_t e : hev)
+    if (e) cudaEventDestroy(e);
+  if (h->h2d) cudaStreamDestroy(h->h2d);
+  if (h->d2h) cudaStreamDestroy(h->d2h);
   cudaFree(h->wo16);
   cudaFree(h->wqkvT16);
   cudaFree(h->woT);
@@ -571,6 +594,17 @@ const char* mot_status_string(mot_status s) {
     case MOT_ERR_TIMEOUT: return "bounded in-kernel wait expired";
   }
   return "unknown status";
+}
+
+mot_status mot_attn_query_host_staging(const mot_attn_config* cfg, int32_t batch, int32_t img_tokens,
+                                       int32_t prefix_max, size_t* staging_bytes) {
+  mot_status st = check_config(cfg);
+  if (st != MOT_OK) return st;
+  if (!staging_bytes || batch <= 0 || img_tokens <= 0 || prefix_max < 0) return MOT_ERR_INVALID_ARGUMENT;
+  if (batch > cfg->max_batch || img_tokens > cfg->max_img_tokens || prefix_max > cfg->max_prefix)
+    return MOT_ERR_UNSUPPORTED_SHAPE;
+  *staging_bytes = 2 * host_staging(*cfg, batch, img_tokens, prefix_max).slot;
+  return MOT_OK;
 }
 
 mot_status mot_attn_query_sizes(const mot_attn_config* cfg, int32_t batch, int32_t img_tokens, int32_t prefix_max,
@@ -1282,6 +1316,94 @@ void* noalloc_scratch_address() {
   return g_noalloc_ptr[dev];
 }
 }  // namespace
+
+extern "C" mot_status mot_attn_forward_host(mot_attn_t h, int32_t steps, const void* const* x_host, int32_t B,
+                                            int32_t N, const void* const* k_cache_host,
+                                            const void* const* v_cache_host, const int32_t* prefix_len, int32_t P,
+                                            void* const* y_host, void* staging, size_t staging_bytes,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!h || steps <= 0 || !x_host || !y_host || !prefix_len || !staging || !workspace)
+    return MOT_ERR_INVALID_ARGUMENT;
+  const mot_attn_config& c = h->cfg;
+  if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
+  if (B > c.max_batch || N > c.max_img_tokens || P > c.max_prefix) return MOT_ERR_UNSUPPORTED_SHAPE;
+  if (P > 0 && (!k_cache_host || !v_cache_host)) return MOT_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < steps; ++i) {
+    if (!x_host[i] || !y_host[i]) return MOT_ERR_INVALID_ARGUMENT;
+    if (P > 0 && (!k_cache_host[i] || !v_cache_host[i])) return MOT_ERR_INVALID_ARGUMENT;
+  }
+  for (int b = 0; b < B; ++b)
+    if (prefix_len[b] < 0 || prefix_len[b] > P) return MOT_ERR_INVALID_ARGUMENT;
+  if (!aligned16(staging) || !aligned16(workspace)) return MOT_ERR_ALIGNMENT;
+  const HostStaging hs = host_staging(c, B, N, P);
+  if (staging_bytes < 2 * hs.slot) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  const Layout L = make_layout(c, B, N, P, false);
+  if (workspace_bytes < L.fwd_scratch + L.act_bytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  if (!h->h2d) {
+    bool ok = cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->hev_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int s = 0; s < 2 && ok; ++s)
+      ok = cudaEventCreateWithFlags(&h->hev_in[s], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->hev_comp[s], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->hev_out[s], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return MOT_ERR_CUDA;  // what was made is released with the handle
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  auto note = [&err](cudaError_t e) {
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    return err == cudaSuccess;
+  };
+  // both copy streams start after the work already on the caller's stream
+  note(cudaEventRecord(h->hev_start, st));
+  note(cudaStreamWaitEvent(h->h2d, h->hev_start, 0));
+  note(cudaStreamWaitEvent(h->d2h, h->hev_start, 0));
+  const size_t xb = static_cast<size_t>(B) * N * c.hidden * 2;
+  const size_t kvb = static_cast<size_t>(B) * c.n_kv_heads * P * c.head_dim * 2;
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  mot_status status = MOT_OK;
+  for (int i = 0; i < steps && err == cudaSuccess; ++i) {
+    const int s = i & 1;
+    uint8_t* slot = base + s * hs.slot;
+    void* xd = slot;
+    void* yd = slot + hs.x;
+    void* kd = slot + 2 * hs.x;
+    void* vd = slot + 2 * hs.x + hs.kv;
+    // copy-in; the slot's inputs were last read by the layer of call i-2
+    if (i >= 2) note(cudaStreamWaitEvent(h->h2d, h->hev_comp[s], 0));
+    note(cudaMemcpyAsync(xd, x_host[i], xb, cudaMemcpyHostToDevice, h->h2d));
+    if (P > 0) {
+      note(cudaMemcpyAsync(kd, k_cache_host[i], kvb, cudaMemcpyHostToDevice, h->h2d));
+      note(cudaMemcpyAsync(vd, v_cache_host[i], kvb, cudaMemcpyHostToDevice, h->h2d));
+    }
+    note(cudaEventRecord(h->hev_in[s], h->h2d));
+    // the layer, once its inputs landed and call i-2's y has left the slot
+    note(cudaStreamWaitEvent(st, h->hev_in[s], 0));
+    if (i >= 2) note(cudaStreamWaitEvent(st, h->hev_out[s], 0));
+    if (err != cudaSuccess) break;
+    status = mot_attn_forward(h, xd, B, N, P > 0 ? kd : nullptr, P > 0 ? vd : nullptr, prefix_len, P, yd, nullptr,
+                              nullptr, 0, workspace, workspace_bytes, stream);
+    if (status != MOT_OK) break;
+    note(cudaEventRecord(h->hev_comp[s], st));
+    // copy-out
+    note(cudaStreamWaitEvent(h->d2h, h->hev_comp[s], 0));
+    note(cudaMemcpyAsync(y_host[i], yd, xb, cudaMemcpyDeviceToHost, h->d2h));
+    note(cudaEventRecord(h->hev_out[s], h->d2h));
+  }
+  // on every path the caller's stream ends after all copies enqueued so far
+  // (each copy stream runs in order, so its latest event covers the rest)
+  cudaError_t e1 = cudaEventRecord(h->hev_out[0], h->d2h);
+  cudaError_t e2 = cudaStreamWaitEvent(st, h->hev_out[0], 0);
+  cudaError_t e3 = cudaEventRecord(h->hev_in[0], h->h2d);
+  cudaError_t e4 = cudaStreamWaitEvent(st, h->hev_in[0], 0);
+  note(e1);
+  note(e2);
+  note(e3);
+  note(e4);
+  if (status != MOT_OK) return status;
+  return err == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+}
 
 extern "C" mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int32_t B, int32_t N,
                                                const void* k_cache, const void* v_cache,

@@ -86,6 +86,34 @@ def mot_attn_backward(h, dy, x, batch, img_tokens, k_cache, v_cache, prefix_len:
           "mot_attn_backward")
 
 
+def mot_attn_query_host_staging(cfg: MotAttnConfig, batch: int, img_tokens: int, prefix_max: int) -> int:
+    n = c_size_t(0)
+    check(lib().mot_attn_query_host_staging(byref(cfg), batch, img_tokens, prefix_max, byref(n)),
+          "mot_attn_query_host_staging")
+    return n.value
+
+
+def _host_ptrs(ts: Sequence[Optional[torch.Tensor]]):
+    for t in ts:
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("host buffers must be contiguous CPU tensors")
+    return (c_void_p * len(ts))(*[t.data_ptr() if t is not None else None for t in ts])
+
+
+def mot_attn_forward_host(h, xs, batch, img_tokens, k_caches, v_caches, prefix_len: Sequence[int], prefix_max,
+                          ys, staging, workspace, stream=None) -> None:
+    steps = len(xs)
+    if len(ys) != steps or (k_caches is not None and len(k_caches) != steps) or \
+            (v_caches is not None and len(v_caches) != steps):
+        raise ValueError("one x, y (and cache) buffer per call")
+    pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
+    kc = _host_ptrs(k_caches) if k_caches is not None else None
+    vc = _host_ptrs(v_caches) if v_caches is not None else None
+    check(lib().mot_attn_forward_host(h, steps, _host_ptrs(xs), batch, img_tokens, kc, vc, pl, prefix_max,
+                                      _host_ptrs(ys), _ptr(staging), staging.numel(), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "mot_attn_forward_host")
+
+
 def mot_attn_merge_lora(h, w_q_out, w_k_out, w_v_out, w_o_out, stream=None) -> None:
     check(lib().mot_attn_merge_lora(h, _ptr(w_q_out), _ptr(w_k_out), _ptr(w_v_out), _ptr(w_o_out),
                                     _stream(stream)), "mot_attn_merge_lora")
@@ -196,6 +224,24 @@ class MotAttnLayer:
             workspace = self.workspace(B, N, P, x.device)
         mot_attn_forward(self.handle, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, saved, workspace, stream)
         return y
+
+    def host_staging(self, batch, img_tokens, prefix_max, device="cuda"):
+        n = mot_attn_query_host_staging(self.cfg, batch, img_tokens, prefix_max)
+        return torch.empty(n, dtype=torch.uint8, device=device)
+
+    def forward_host(self, xs, k_caches, v_caches, prefix_len, ys, staging=None, workspace=None, stream=None):
+        """Inference forwards over host buffers (one x, k_cache, v_cache, y
+        per call; pinned for overlap): copies in, layer and copies out are
+        pipelined over two device staging slots. Asynchronous: the y buffers
+        are complete once `stream` has finished the enqueued work."""
+        B, N, d = xs[0].shape
+        P = k_caches[0].shape[2] if k_caches is not None else 0
+        if staging is None:
+            staging = self.host_staging(B, N, P)
+        if workspace is None:
+            workspace = self.workspace(B, N, P)
+        mot_attn_forward_host(self.handle, xs, B, N, k_caches, v_caches, prefix_len, P, ys, staging, workspace,
+                              stream)
 
     def backward(self, dy, x, k_cache, v_cache, prefix_len, saved, dx=None, dx_f32=None, d_a=None, d_b=None,
                  accumulate=False, workspace=None, stream=None):

@@ -95,3 +95,27 @@ def test_forward_backward_reject_null_handle(L):
     assert L.mot_attn_merge_lora(None, None, None, None, None, None) == _abi.MOT_ERR_INVALID_ARGUMENT
     assert L.mot_attn_last_launch_count(None) == 0
     L.mot_attn_destroy(None)
+
+
+def test_host_staging_size_host_only(L):
+    cfg = make_config(lora_rank=32, lora_alpha=32, max_batch=2, max_img_tokens=4096, max_prefix=400)
+    n = c_size_t()
+    assert L.mot_attn_query_host_staging(byref(cfg), 2, 4096, 400, byref(n)) == _abi.MOT_OK
+    # two slots of x and y (2*4096*4096 bf16 each) and the two caches (2*8*400*128 bf16 each)
+    x = 2 * 4096 * 4096 * 2
+    kv = 2 * 8 * 400 * 128 * 2
+    assert n.value == 2 * (2 * x + 2 * kv)
+    assert L.mot_attn_query_host_staging(byref(cfg), 2, 4096, 0, byref(n)) == _abi.MOT_OK
+    assert n.value == 2 * 2 * x
+    assert L.mot_attn_query_host_staging(byref(cfg), 3, 4096, 400, byref(n)) == _abi.MOT_ERR_UNSUPPORTED_SHAPE
+    assert L.mot_attn_query_host_staging(byref(cfg), 2, 4096, 400, None) == _abi.MOT_ERR_INVALID_ARGUMENT
+
+
+def test_forward_host_rejects_bad_arguments_before_cuda(L):
+    one = (c_void_p * 1)(None)
+    pl = (ctypes.c_int32 * 1)(0)
+    # no handle, no calls, null buffer arrays: rejected on the host
+    assert L.mot_attn_forward_host(None, 1, one, 1, 16, None, None, pl, 0, one, None, 0, None, 0, None) \
+        == _abi.MOT_ERR_INVALID_ARGUMENT
+    assert L.mot_attn_forward_host(None, 0, one, 1, 16, None, None, pl, 0, one, None, 0, None, 0, None) \
+        == _abi.MOT_ERR_INVALID_ARGUMENT
