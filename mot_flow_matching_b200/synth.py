@@ -133,6 +133,37 @@ def make_inputs(wl: Workload, seed_base: int, with_dy: Optional[bool] = None,
     return out
 
 
+# the gen-tower MLP's tensors (the next block of the same decoder layer);
+# indices apart from the attention layer's
+_MLP_TENSOR_INDEX = {
+    "x": 40, "w_gate": 41, "w_up": 42, "w_down": 43, "a_gate": 44, "a_up": 45, "a_down": 46,
+    "b_gate": 47, "b_up": 48, "b_down": 49, "dy": 50,
+}
+
+
+def make_mlp_inputs(tokens: int, hidden: int, inter: int, lora_rank: int, seed_base: int,
+                    with_dy: bool = False) -> Dict[str, torch.Tensor]:
+    """CPU bf16 tensors for one gen-tower SwiGLU MLP call, with the same
+    distributions as the attention layer's: x, dy [tokens, hidden];
+    w_gate, w_up [inter, hidden]; w_down [hidden, inter]; a_gate, a_up
+    [r, hidden]; a_down [r, inter]; b_gate, b_up [inter, r]; b_down [hidden, r]."""
+    s = lambda name: seed_base + _MLP_TENSOR_INDEX[name]
+    r = lora_rank
+    out = {
+        "x": _draw((tokens, hidden), 1.0, 0.0, s("x")),
+        "w_gate": _draw((inter, hidden), 0.02, 0.0, s("w_gate")),
+        "w_up": _draw((inter, hidden), 0.02, 0.0, s("w_up")),
+        "w_down": _draw((hidden, inter), 0.02, 0.0, s("w_down")),
+    }
+    if r > 0:
+        for name, shape in {"a_gate": (r, hidden), "a_up": (r, hidden), "a_down": (r, inter),
+                            "b_gate": (inter, r), "b_up": (inter, r), "b_down": (hidden, r)}.items():
+            out[name] = _draw(shape, 1.0 / 16.0 if name.startswith("a_") else 0.01, 0.0, s(name))
+    if with_dy:
+        out["dy"] = _draw((tokens, hidden), 1.0, 0.0, s("dy"))
+    return out
+
+
 def workload_inputs(index: int, with_dy: Optional[bool] = None, shard: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(WORKLOADS[index], 1000 * index, with_dy, shard)
 

@@ -1,5 +1,6 @@
-"""Regression pin: the oracle still reproduces tests/golden/tiny_layer.json
-(written by tests/golden/make_golden.py from the oracle alone)."""
+"""Regression pins: the oracles still reproduce tests/golden/tiny_layer.json
+and tiny_mlp.json (written by tests/golden/make_golden.py from the oracles
+alone)."""
 import json
 import os
 
@@ -15,4 +16,13 @@ def test_oracle_matches_stored_tiny_case():
         ref = json.load(f)
     now = compute()
     for key in ("y", "dx", "dA_q", "dB_o"):
+        np.testing.assert_allclose(np.array(now[key]), np.array(ref[key]), rtol=1e-12, atol=1e-13)
+
+
+def test_mlp_oracle_matches_stored_tiny_case():
+    from tests.golden.make_golden import compute_mlp
+    with open(os.path.join(HERE, "golden", "tiny_mlp.json")) as f:
+        ref = json.load(f)
+    now = compute_mlp()
+    for key in ("y", "dx", "dA_up", "dB_down"):
         np.testing.assert_allclose(np.array(now[key]), np.array(ref[key]), rtol=1e-12, atol=1e-13)
