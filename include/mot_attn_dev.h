@@ -76,6 +76,14 @@ mot_status mot_dev_stage_timeline(mot_attn_t h, int32_t* ids, float* t0_ms, floa
  * x, y device f32 [n], n even, x in [-125, 8]. For accuracy tests. */
 mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream);
 
+/* Failure-detection check: enqueue on `stream` one kernel whose single wait
+ * is on a barrier nothing ever completes, through the bounded wait all the
+ * kernels use. The wait gives up after its limit (2 s), latches the timeout
+ * in the handle's device status and the kernel exits normally, so the next
+ * mot_attn_get_device_status returns MOT_ERR_TIMEOUT and the handle and the
+ * context stay usable. For tests. */
+mot_status mot_dev_wait_probe(mot_attn_t h, void* stream);
+
 /* Static name of a stage id ("qkv_gemm", "attn_fwd", ...; "?" if unknown). */
 const char* mot_dev_stage_name(int32_t id);
 

@@ -66,6 +66,7 @@ SIGNATURES = {
     "mot_dev_profile": (c_int32, [c_void_p, c_int32]),
     "mot_dev_stage_times": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), c_int32, POINTER(c_int32)]),
     "mot_dev_stage_name": (c_char_p, [c_int32]),
+    "mot_dev_wait_probe": (c_int32, [c_void_p, c_void_p]),
     "mot_dev_stage_timeline": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), POINTER(c_float), c_int32,
                                          POINTER(c_int32)]),
     "mot_dev_saved_layout": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32, POINTER(c_size_t),

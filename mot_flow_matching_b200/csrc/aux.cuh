@@ -160,6 +160,24 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
   if (i < npairs) exp2_poly2(y[2 * i], y[2 * i + 1], x[2 * i], x[2 * i + 1]);
 }
 
+// Failure-detection check of the bounded waits: one thread waits on an
+// mbarrier that nothing ever arrives on, through the same bounded wait every
+// kernel uses, so the wait gives up after its limit, latches DEV_ERR_TIMEOUT
+// in `status` and the kernel exits normally (no trap, no fault).
+__global__ void wait_probe_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitGuard wg{&abort_flag, status};
+  if (threadIdx.x == 0) mbar_wait(&bar, 0u, wg);  // phase 0 never completes
+  __syncthreads();
+}
+
 // f32 copy of a bf16 vector (norm gains)
 __global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

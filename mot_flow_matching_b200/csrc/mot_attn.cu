@@ -1550,6 +1550,12 @@ mot_status mot_dev_stage_timeline(mot_attn_t h, int32_t* ids, float* t0_ms, floa
   return MOT_OK;
 }
 
+mot_status mot_dev_wait_probe(mot_attn_t h, void* stream) {
+  if (!h) return MOT_ERR_INVALID_ARGUMENT;
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->status);
+  return cudaGetLastError() == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
+}
+
 const char* mot_dev_stage_name(int32_t id) {
   if (id >= 0 && id < static_cast<int32_t>(sizeof(kStageNames) / sizeof(kStageNames[0]))) return kStageNames[id];
   return "?";

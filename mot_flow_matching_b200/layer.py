@@ -165,6 +165,10 @@ def mot_dev_exp2_poly(x, y, stream=None) -> None:
     check(lib().mot_dev_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "mot_dev_exp2_poly")
 
 
+def mot_dev_wait_probe(h, stream=None) -> None:
+    check(lib().mot_dev_wait_probe(h, _stream(stream)), "mot_dev_wait_probe")
+
+
 def mot_dev_profile(h, enable: bool) -> None:
     check(lib().mot_dev_profile(h, int(bool(enable))), "mot_dev_profile")
 
