@@ -139,6 +139,36 @@ def gqa_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
     return o, probs, lse
 
 
+def merge_attention_partials(partials: Sequence):
+    """Combine partial attention results over disjoint key ranges.
+
+    Each partial is (o_s, lse_s): softmax attention restricted to one key
+    range (o_s [..., n, dh] normalised within the range, lse_s [..., n] its
+    natural-log normaliser). Over the union of the ranges
+        lse = log sum_s exp(lse_s),   o = sum_s exp(lse_s - lse) o_s,
+    since exp(lse_s - lse) is the share of the total softmax mass that range s
+    holds. This is the split-KV merge the flash-attention kernels of
+    "SenseNova-U1" (vLLM-Omni recipe, measured kernel table) rest on.
+    """
+    lses = np.stack([np.asarray(l, dtype=np.float64) for _, l in partials])
+    m = lses.max(axis=0)
+    lse = m + np.log(np.sum(np.exp(lses - m), axis=0))
+    o = sum(np.exp(l - lse)[..., None] * np.asarray(o_s, dtype=np.float64) for o_s, l in partials)
+    return o, lse
+
+
+def gqa_attention_split_kv(q: np.ndarray, k: np.ndarray, v: np.ndarray, bounds: Sequence[int]):
+    """gqa_attention over the keys cut at ``bounds`` (0 < b_1 < ... < L,
+    contiguous ranges [b_i, b_{i+1})), each range computed on its own and the
+    partials merged by merge_attention_partials. Returns (o, lse)."""
+    cuts = [0] + [int(b) for b in bounds] + [k.shape[1]]
+    parts = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        o_s, _, lse_s = gqa_attention(q, k[:, lo:hi], v[:, lo:hi])
+        parts.append((o_s, lse_s))
+    return merge_attention_partials(parts)
+
+
 def gqa_attention_backward(do: np.ndarray, q: np.ndarray, k: np.ndarray, v: np.ndarray,
                            o: np.ndarray, probs: np.ndarray):
     """Backward of gqa_attention; returns (dq, dk, dv) with dk, dv summed over
