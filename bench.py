@@ -87,7 +87,10 @@ def stage_work(wl, stage):
     if stage == "lora_down_o":
         return 2.0 * M * Hq * dh * r, 2.0 * (M * Hq * dh + r * Hq * dh + M * r)
     if stage == "build_kv":
-        return 0.0, 2.0 * 2 * B * Hkv * P * dh * 2
+        # cache prefix rows in (bf16) and out (f16), zero tail rows out, LoRA f16 copies in and out
+        tail = (-(P + N)) % 128
+        lora = 2.0 * 2 * r * (Hq * dh + hid + qkv)
+        return 0.0, 2.0 * 2 * B * Hkv * P * dh * 2 + 2.0 * 2 * B * Hkv * tail * dh + lora
     if stage == "cvt_lora_o":
         return 0.0, 2.0 * 2 * r * (Hq * dh + hid + qkv)
     # backward (LoRA training): base, gains and cache frozen
@@ -221,6 +224,34 @@ def run_reference(args):
     return 0
 
 
+def run_once_mlp(args):
+    """Two warm MLP calls (forward, or forward + backward with --train) of
+    an MLP workload (the target of ncu captures)."""
+    import torch
+    from mot_flow_matching_b200 import synth
+    from mot_flow_matching_b200.mlp import MotMlp
+    wl = synth.MLP_WORKLOADS[args.workload]
+    t = synth.mlp_workload_inputs(args.workload, with_dy=args.train)
+    td = {k: v.cuda() for k, v in t.items()}
+    w = {k: td[k] for k in td if k.startswith(("w_", "a_", "b_"))}
+    m = MotMlp(w, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_tokens=wl.tokens,
+               enable_backward=args.train, hidden=wl.hidden, intermediate=wl.inter)
+    sv = m.new_saved(wl.tokens) if args.train else None
+    names = ("gate", "up", "down")
+    d_a = [torch.zeros(td["a_" + n].shape, device="cuda") for n in names] if args.train else None
+    d_b = [torch.zeros(td["b_" + n].shape, device="cuda") for n in names] if args.train else None
+    for _ in range(2):
+        y = m.forward(td["x"], saved=sv)
+        if args.train:
+            m.backward(td["dy"], td["x"], sv, d_a=d_a, d_b=d_b)
+    torch.cuda.synchronize()
+    status = m.device_status()
+    m.close()
+    print(json.dumps({"once": wl.name, "train": bool(args.train), "status": status,
+                      "y_abs_mean": float(y.float().abs().mean())}))
+    return 0 if status == 0 else 1
+
+
 def run_once(args):
     """One warm forward of a workload (the target of ncu captures)."""
     import torch
@@ -228,6 +259,8 @@ def run_once(args):
     from mot_flow_matching_b200 import synth
     from mot_flow_matching_b200.layer import MotAttnLayer
     build_mod.build()
+    if args.mlp:
+        return run_once_mlp(args)
     wl = synth.WORKLOADS[args.workload]
     t = synth.workload_inputs(args.workload)
     td = {k: (v.cuda() if k != "prefix_len" else v) for k, v in t.items()}
@@ -338,6 +371,143 @@ def train_steps(bundle, dev, flush, stream, args, world):
             "bwd_pct_of_bf16_peak": 100.0 * bwd_flops / (b / 1e3) / 1e12 / peaks["bf16_tflops"],
             "bwd_algorithmic_gflop": bwd_flops / 1e9, "gpu_launches": launches * world, "stages": per,
             "bwd_timeline_ms": timeline}
+
+
+MLP_INDEX = 2        # the MLP over the 2048^2 CFG call's 8192 tokens
+MLP_TRAIN_INDEX = 4  # the MLP training step over 4096 tokens
+
+
+def mlp_flops(wl):
+    """Algorithmic FLOPs of one MLP forward (gate/up, down, LoRA down and up)."""
+    T, d, I, r = wl.tokens, wl.hidden, wl.inter, wl.lora_rank
+    return 6.0 * T * d * I + 2.0 * T * r * (2 * d + 2 * I + I + d)
+
+
+def mlp_steps(dev, flush, stream, args, world):
+    """The SwiGLU MLP: forward over the 2048^2 CFG tokens, forward + backward
+    over the training tokens; CUDA events on the launching stream, L2 flushed
+    before every step; per-launch times from separate passes."""
+    import torch
+    from mot_flow_matching_b200 import dp, synth
+    from mot_flow_matching_b200.mlp import MotMlp, mot_dev_mlp_profile, mot_dev_mlp_stage_times
+    peaks, _ = load_peaks()
+    out = {}
+    for key, idx in (("forward", MLP_INDEX), ("train", MLP_TRAIN_INDEX)):
+        wl = synth.MLP_WORKLOADS[idx]
+        t = synth.mlp_workload_inputs(idx)
+        td = {k: v.to(dev) for k, v in t.items()}
+        w = {k: td[k] for k in td if k.startswith(("w_", "a_", "b_"))}
+        m = MotMlp(w, lora_rank=wl.lora_rank, lora_alpha=wl.lora_alpha, max_tokens=wl.tokens,
+                   enable_backward=wl.train, hidden=wl.hidden, intermediate=wl.inter)
+        x = td["x"]
+        y = torch.empty_like(x)
+        ws = m.workspace(wl.tokens, dev)
+        train = wl.train
+        sv = m.new_saved(wl.tokens, dev) if train else None
+        names = ("gate", "up", "down")
+        d_a = [torch.zeros(td["a_" + n].shape, device=dev) for n in names] if train else None
+        d_b = [torch.zeros(td["b_" + n].shape, device=dev) for n in names] if train else None
+        dx = torch.empty_like(x)
+
+        def step(ev=None):
+            if ev:
+                ev[0].record(stream)
+            m.forward(x, y=y, saved=sv, workspace=ws)
+            if ev:
+                ev[1].record(stream)
+            if train:
+                m.backward(td["dy"], x, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
+                if ev:
+                    ev[2].record(stream)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        dp.barrier(world)
+        steps = max(3, args.steps // 2)
+        f_ms, b_ms = [], []
+        for _ in range(steps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            step(ev)
+            ev[2 if train else 1].synchronize()
+            f_ms.append(ev[0].elapsed_time(ev[1]))
+            if train:
+                b_ms.append(ev[1].elapsed_time(ev[2]))
+        stages = {}
+        mot_dev_mlp_profile(m.handle, True)
+        for _ in range(steps):
+            flush.zero_()
+            m.forward(x, y=y, saved=sv, workspace=ws)
+            for n, v in mot_dev_mlp_stage_times(m.handle):
+                stages.setdefault(n, []).append(v)
+            if train:
+                m.backward(td["dy"], x, sv, dx=dx, d_a=d_a, d_b=d_b, accumulate=True, workspace=ws)
+                for n, v in mot_dev_mlp_stage_times(m.handle):
+                    stages.setdefault(n, []).append(v)
+        mot_dev_mlp_profile(m.handle, False)
+        assert m.device_status() == 0
+        m.close()
+        f = dp.max_over_ranks(statistics.mean(f_ms), world, dev)
+        fl = mlp_flops(wl)
+        rec = {"workload": wl.name, "tokens": wl.tokens, "intermediate": wl.inter, "lora_rank": wl.lora_rank,
+               "fwd_ms": f, "fwd_tflops": fl / (f / 1e3) / 1e12,
+               "fwd_frac_of_bf16_peak": fl / (f / 1e3) / 1e12 / peaks["bf16_tflops"],
+               "tokens_per_s": world * wl.tokens / (f / 1e3),
+               "stages_ms": {n: sum(v) / steps for n, v in stages.items()}}
+        if train:
+            b = dp.max_over_ranks(statistics.mean(b_ms), world, dev)
+            bfl = 6.0 * wl.tokens * wl.hidden * wl.inter + 2.0 * wl.tokens * wl.lora_rank * 4 * (wl.hidden + wl.inter)
+            rec.update({"bwd_ms": b, "bwd_tflops": bfl / (b / 1e3) / 1e12,
+                        "bwd_frac_of_bf16_peak": bfl / (b / 1e3) / 1e12 / peaks["bf16_tflops"]})
+        out[key] = rec
+    return out
+
+
+def sustained_steps(bundle, dev, stream, args, world, local):
+    """Back-to-back forwards of one workload for at least args.sustained_s
+    seconds under one pair of CUDA events, SM clock sampled throughout;
+    reported against the sustained bf16 peak and normalised by the clock."""
+    import torch
+    from mot_flow_matching_b200 import dp
+    wl, _, td, layer = bundle
+    x, kc, vc = td["x"], td["k_cache"], td["v_cache"]
+    pl = [int(v) for v in td["prefix_len"]]
+    y = torch.empty_like(x)
+    ws = layer.workspace(wl.batch, wl.img_tokens, wl.prefix, dev)
+    for _ in range(args.warmup):
+        layer.forward(x, kc, vc, pl, y=y, workspace=ws)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(20):
+        layer.forward(x, kc, vc, pl, y=y, workspace=ws)
+    e1.record(stream)
+    e1.synchronize()
+    n = max(20, int(args.sustained_s * 1e3 / (e0.elapsed_time(e1) / 20)))
+    dp.barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(n):
+        layer.forward(x, kc, vc, pl, y=y, workspace=ws)
+    e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    total = dp.max_over_ranks(e0.elapsed_time(e1), world, dev)
+    layer.close()
+    peaks, kind = load_peaks()
+    fl = sum(stage_work(wl, s)[0] for s in ("lora_down_qkv", "qkv_gemm", "attn_fwd", "lora_down_o", "o_gemm"))
+    ms = total / n
+    tf = fl / (ms / 1e3) / 1e12
+    out = {"workload": wl.name, "steps": n, "seconds": total / 1e3, "ms_per_step": ms, "tflops": tf,
+           "peak": peaks["bf16_tflops_sustained"], "frac": tf / peaks["bf16_tflops_sustained"],
+           "peak_source": f"{kind} (sustained)", "clocks": clk,
+           "value": dp.aggregate_rate(wl.batch * wl.img_tokens, n, total, world)}
+    if clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        # the same time at the maximum SM clock, if the layer scaled with it
+        out["ms_per_step_at_max_clock"] = ms * clk["sm_mhz"] / clk["sm_max_mhz"]
+    return out
 
 
 def run_ours(args):
@@ -503,15 +673,43 @@ def run_ours(args):
         # the edit workload: adapters baked into the base (merge at load), then rank-0 calls
         wl3, _, td3, layer3 = make(EDIT_INDEX)
         merged = {n: torch.empty_like(td3["w_" + n]) for n in ("q", "k", "v", "o")}
+        # the one-off merge at load, timed on its own (flushed L2)
+        torch.cuda.synchronize(dev)
+        flush.zero_()
+        em0, em1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        em0.record(stream)
         layer3.merge_lora(merged["q"], merged["k"], merged["v"], merged["o"])
+        em1.record(stream)
+        em1.synchronize()
+        merge_ms = em0.elapsed_time(em1)
         ms3, _, _ = device_steps(wl3, td3, layer3, max(3, args.steps // 2), args.warmup, False)
         max3 = dp.max_over_ranks(sum(ms3), world, dev)
         fl3 = 4.0 * wl3.batch * wl3.dims.n_q_heads * wl3.img_tokens * (wl3.prefix + wl3.img_tokens) * wl3.dims.head_dim
         fl3 += 2.0 * wl3.batch * wl3.img_tokens * wl3.dims.hidden * (
             (wl3.dims.n_q_heads + 2 * wl3.dims.n_kv_heads) * wl3.dims.head_dim + wl3.dims.n_q_heads * wl3.dims.head_dim)
         also = [also, {"workload": wl3.name, "value": dp.aggregate_rate(wl3.batch * wl3.img_tokens, len(ms3), max3, world),
-                       "ms_per_step": max3 / len(ms3), "tflops": fl3 / (max3 / len(ms3) / 1e3) / 1e12}]
+                       "ms_per_step": max3 / len(ms3), "tflops": fl3 / (max3 / len(ms3) / 1e3) / 1e12,
+                       "merge_lora_ms": merge_ms}]
         layer3.close()
+        # the 512^2 single-branch workload (the smallest; latency-bound)
+        wl0, _, td0, layer0 = make(0)
+        ms0, st0, _ = device_steps(wl0, td0, layer0, max(3, args.steps // 2), args.warmup, True)
+        max0 = dp.max_over_ranks(sum(ms0), world, dev)
+        fl0 = sum(stage_work(wl0, n)[0] for n in st0)
+        also.insert(0, {"workload": wl0.name, "value": dp.aggregate_rate(wl0.batch * wl0.img_tokens, len(ms0), max0, world),
+                        "ms_per_step": max0 / len(ms0), "tflops": fl0 / (max0 / len(ms0) / 1e3) / 1e12,
+                        "attn_ms": sum(st0.get("attn_fwd", [0.0])) / len(ms0)})
+        layer0.close()
+
+    # the gen-tower SwiGLU MLP on the same token counts
+    mlp = None
+    if not args.skip_mlp:
+        mlp = mlp_steps(dev, flush, stream, args, world)
+
+    # sustained: back-to-back 2048^2 CFG forwards for >= 2 s, clocks sampled
+    sustained = None
+    if args.sustained_s > 0:
+        sustained = sustained_steps(make(WORKLOAD_INDEX), dev, stream, args, world, local)
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
@@ -519,13 +717,13 @@ def run_ours(args):
         stage_summary = {}
         for name, v in stages.items():
             fl, by = stage_work(wl, name)
-            avg = statistics.mean(v)
+            avg = sum(v) / args.steps  # per step (a stage may launch more than once per step)
             stage_summary[name] = {"ms": avg, "share": sum(v) / sum(sum(x) for x in stages.values()),
                                    "tflops": fl / (avg / 1e3) / 1e12 if fl else None,
                                    "gbs": by / (avg / 1e3) / 1e9}
         top = max(stages, key=lambda n: sum(stages[n]))
         fl, by = stage_work(wl, top)
-        avg_top = statistics.mean(stages[top])
+        avg_top = sum(stages[top]) / args.steps
         if fl > 0:
             achieved, peak, unit, bound = fl / (avg_top / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
         else:
@@ -564,9 +762,40 @@ def run_ours(args):
             "clocks": clk,
             "also": also,
             "train": train,
+            "mlp": mlp,
+            "sustained": sustained,
         }
         print(json.dumps(line), flush=True)
     layer.close()
+    dp.finish(world)
+    return 0
+
+
+def run_rank_check(args):
+    """The rank plumbing of run_ours on CPU (gloo): group, per-rank data
+    shards, barrier, max over ranks of each rank's time and the whole-job
+    rate; rank 0 prints one JSON line. For the multi-process CPU tests."""
+    import torch
+    from mot_flow_matching_b200 import dp, synth
+    world, rank, local = dp.world_info()
+    dp.init_group(world, "gloo", timeout_s=60)
+    wl = synth.tiny_workload()
+    t = synth.make_inputs(wl, 77, shard=rank)
+    dp.barrier(world)
+    t0 = time.perf_counter()
+    ref = sum(float(v.float().sum()) for k, v in t.items() if k != "prefix_len")
+    ms = (time.perf_counter() - t0) * 1e3 + 1.0
+    total = dp.max_over_ranks(ms * args.steps, world)
+    sums = torch.tensor([ref], dtype=torch.float64)
+    gathered = [torch.zeros_like(sums) for _ in range(world)]
+    if world > 1:
+        torch.distributed.all_gather(gathered, sums)
+    else:
+        gathered = [sums]
+    if rank == 0:
+        print(json.dumps({"check": "ranks", "n_gpus": world, "local_rank": local, "steps": args.steps,
+                          "value": dp.aggregate_rate(wl.batch * wl.img_tokens, args.steps, total, world),
+                          "shard_sums": [float(g[0]) for g in gathered]}), flush=True)
     dp.finish(world)
     return 0
 
@@ -580,11 +809,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-also", action="store_true")
     ap.add_argument("--skip-train", action="store_true")
+    ap.add_argument("--skip-mlp", action="store_true")
+    ap.add_argument("--sustained-s", type=float, default=2.0,
+                    help="seconds of back-to-back forwards for the sustained figure (0: skip)")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--once", action="store_true", help="one warm forward, no timing (ncu target)")
     ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX)
     ap.add_argument("--train", action="store_true", help="with --once: forward keeping activations + backward")
+    ap.add_argument("--mlp", action="store_true", help="with --once: the gen-tower MLP instead of the attention")
+    ap.add_argument("--check-ranks", action="store_true",
+                    help="CPU check of the rank plumbing (gloo): spawn/launcher handling, shards, max over ranks")
     args = ap.parse_args()
     if args.once:
         return run_once(args)
@@ -592,6 +827,18 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    # --gpus N means N ranks, one per GPU: as launched by torchrun (whose
+    # WORLD_SIZE must then be N), or started here when no launcher did
+    from mot_flow_matching_b200 import dp
+    try:
+        how = dp.check_world(args.gpus)
+    except ValueError as e:
+        print(f"bench.py: {e}", file=sys.stderr)
+        return 2
+    if how == "spawn":
+        return dp.spawn_local_ranks(args.gpus, [sys.executable, os.path.abspath(__file__)] + sys.argv[1:])
+    if args.check_ranks:
+        return run_rank_check(args)
     return run_ours(args)
 
 

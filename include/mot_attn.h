@@ -180,11 +180,14 @@ mot_status mot_attn_merge_lora(mot_attn_t h, void* w_q_out, void* w_k_out, void*
  * (inference only). The scratch lives in one 32 MiB device array inside this
  * library (every GPU that loads the library holds it until process exit);
  * a call whose scratch exceeds 32 MiB returns MOT_ERR_WORKSPACE_TOO_SMALL
- * before anything is enqueued (at hidden 4096, LoRA rank 32 and a 400-token
- * prefix that is about 1400 image tokens in one branch; the workspace_bytes
- * of mot_attn_query_sizes is the exact need).
- * The first call on a device resolves the array's device address on the
- * host; make that first call before any stream capture. All calls share the
+ * before anything is enqueued. The scratch is what an inference forward of
+ * the shape needs (its activations and the f16 copies of the LoRA tensors):
+ * at hidden 4096, 32/8 heads, LoRA rank 32 and a 400-token prefix, up to
+ * about 1450 image tokens in one branch.
+ * The current CUDA device must be the one the handle was created on
+ * (MOT_ERR_INVALID_ARGUMENT otherwise). The first call on a device resolves
+ * the array's device address on the host; make that first call before any
+ * stream capture. All calls share the
  * one array and leave their intermediates in it: calls that overlap on the
  * GPU (other streams, other handles, other threads) race and must be
  * serialised by the caller. Nothing in the array needs to start at zero:

@@ -11,6 +11,7 @@
 #include <stdint.h>
 
 #include "mot_attn.h"
+#include "mot_mlp.h"
 
 #ifdef __cplusplus
 extern "C" {
@@ -84,8 +85,34 @@ mot_status mot_dev_exp2_poly(const float* x, float* y, int32_t n, void* stream);
  * context stay usable. For tests. */
 mot_status mot_dev_wait_probe(mot_attn_t h, void* stream);
 
+/* Split-KV count of the attention forward. The work is one unit per
+ * (branch, query head, pair of 128-query tiles). splits == 0 (the default):
+ * each forward plans from the call's shape (key tiles per branch, units, how
+ * many clusters of S CTAs fit on the GPU at once): the units that fill whole
+ * waves of one CTA per SM run unsplit, and the units of a partly empty last
+ * wave may run split S ways in a second launch. splits in 1..8: every unit
+ * of every later forward cuts its keys into exactly that many contiguous
+ * ranges of whole 128-key tiles, one CTA each, merged in split order
+ * (MOT_ERR_UNSUPPORTED_SHAPE from a forward whose shortest branch has fewer
+ * 128-key tiles than splits; from this call if clusters of that size cannot
+ * be resident). For tests and measurements. */
+mot_status mot_dev_set_attn_splits(mot_attn_t h, int32_t splits);
+
+/* Split count of the split units of the last forward (1 if none was split;
+ * 0 before any forward), and how many units it ran unsplit ahead of them. */
+int32_t mot_dev_last_attn_splits(mot_attn_t h);
+int32_t mot_dev_last_attn_full_units(mot_attn_t h);
+
 /* Static name of a stage id ("qkv_gemm", "attn_fwd", ...; "?" if unknown). */
 const char* mot_dev_stage_name(int32_t id);
+
+/* The same per-launch timing for an MLP handle (mot_mlp.h): enable, then
+ * the last call's launches with their stage ids and durations (ms), and the
+ * stage names ("mlp_gate_up", "mlp_down", ...). Same rules as
+ * mot_dev_profile / mot_dev_stage_times. */
+mot_status mot_dev_mlp_profile(mot_mlp_t h, int32_t enable);
+mot_status mot_dev_mlp_stage_times(mot_mlp_t h, int32_t* ids, float* ms, int32_t max, int32_t* count);
+const char* mot_dev_mlp_stage_name(int32_t id);
 
 #ifdef __cplusplus
 }

@@ -37,6 +37,16 @@ class MotAttnWeights(ctypes.Structure):
                                         "a_o", "b_q", "b_k", "b_v", "b_o")]
 
 
+class MotMlpConfig(ctypes.Structure):
+    _fields_ = [("hidden", c_int32), ("intermediate", c_int32), ("lora_rank", c_int32), ("lora_alpha", c_float),
+                ("max_tokens", c_int32), ("enable_backward", c_int32)]
+
+
+class MotMlpWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("w_gate", "w_up", "w_down", "a_gate", "a_up", "a_down", "b_gate", "b_up",
+                                        "b_down")]
+
+
 # name -> (restype, argtypes); every symbol the headers declare
 SIGNATURES = {
     "mot_attn_query_sizes": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32, POINTER(c_size_t),
@@ -67,10 +77,25 @@ SIGNATURES = {
     "mot_dev_stage_times": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), c_int32, POINTER(c_int32)]),
     "mot_dev_stage_name": (c_char_p, [c_int32]),
     "mot_dev_wait_probe": (c_int32, [c_void_p, c_void_p]),
+    "mot_dev_set_attn_splits": (c_int32, [c_void_p, c_int32]),
+    "mot_dev_last_attn_splits": (c_int32, [c_void_p]),
+    "mot_dev_last_attn_full_units": (c_int32, [c_void_p]),
     "mot_dev_stage_timeline": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), POINTER(c_float), c_int32,
                                          POINTER(c_int32)]),
     "mot_dev_saved_layout": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32, POINTER(c_size_t),
                                        POINTER(c_int32)]),
+    "mot_mlp_query_sizes": (c_int32, [POINTER(MotMlpConfig), c_int32, POINTER(c_size_t), POINTER(c_size_t)]),
+    "mot_mlp_create": (c_int32, [POINTER(MotMlpConfig), POINTER(MotMlpWeights), c_void_p, POINTER(c_void_p)]),
+    "mot_mlp_forward": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p,
+                                  c_size_t, c_void_p]),
+    "mot_mlp_backward": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_size_t, c_void_p, c_void_p,
+                                   POINTER(c_void_p), POINTER(c_void_p), c_int32, c_void_p, c_size_t, c_void_p]),
+    "mot_mlp_get_device_status": (c_int32, [c_void_p, c_void_p]),
+    "mot_mlp_last_launch_count": (c_int32, [c_void_p]),
+    "mot_mlp_destroy": (None, [c_void_p]),
+    "mot_dev_mlp_profile": (c_int32, [c_void_p, c_int32]),
+    "mot_dev_mlp_stage_times": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), c_int32, POINTER(c_int32)]),
+    "mot_dev_mlp_stage_name": (c_char_p, [c_int32]),
 }
 
 _lib = None

@@ -25,6 +25,20 @@
 // round trip). The running max is only raised, and O_t rescaled through
 // TMEM, when a row's max grows by more than 2^8; p <= 256 is exact enough in
 // f16 and the final o = O / l uses the same m as every p it summed.
+//
+// Split-KV: with `splits` = S > 1 the key tiles of one (b, h, query pair) are
+// cut into S contiguous ranges, one per CTA of an S-CTA thread-block cluster.
+// Each CTA ends with an unnormalised partial (O_s, m_s, l_s) of its range; it
+// copies O_s (f32) from TMEM into its own shared memory (the Q and K staging
+// areas, idle by then) and (m_s, l_s) beside it, and after a cluster barrier
+// every CTA merges 256/S of the query rows by reading all S partials through
+// distributed shared memory, in split order 0..S-1:
+//   m = max_s m_s,  l = sum_s 2^(m_s - m) l_s,  o = sum_s 2^(m_s - m) O_s / l,
+//   lse = (m + log2 l) ln 2
+// (the log-sum-exp merge of partial softmax results; the same o and lse as
+// one pass over all keys up to f32 summation order). A second cluster
+// barrier keeps every CTA's shared memory alive until all reads are done.
+// No global scratch, no atomics: the result is deterministic for a given S.
 #pragma once
 
 #include "ptx.cuh"
@@ -33,12 +47,15 @@ namespace mot {
 
 constexpr int kAttnThreads = 576;  // TMA warp, MMA warp, 2 x 8 softmax warps
 constexpr float kLazyRescaleLog2 = 8.0f;
+constexpr int kMaxAttnSplits = 8;  // portable cluster size
 
 struct AttnFwdParams {
   CUtensorMap q_map;  // 3D {dh, N, B*Hq} f16, box {64, 128, 1}
   CUtensorMap k_map;  // 3D {dh, Lcap, B*Hkv} f16, box {64, 128, 1}
   CUtensorMap v_map;  // same as k_map
   int B, N, Hq, Hkv, Lcap, q_pairs;  // q_pairs = ceil(N / 256)
+  int splits;                        // S: key-range splits = cluster size (1..kMaxAttnSplits)
+  int unit0;                         // first (b, h, query pair) unit of this launch
   int plen[kMaxBatch];
   float scale_log2;  // log2(e) / sqrt(dh)
   __half* out;       // [B*N, Hq*dh] token-major
@@ -52,7 +69,12 @@ struct AttnSmem {
   static constexpr uint32_t kK = kQ + 2 * kTile;
   static constexpr uint32_t kV = kK + 2 * kTile;
   static constexpr uint32_t kXch = kV + 2 * kTile;  // [2 tiles][2 buffers][2 halves][128] f32
-  static constexpr uint32_t kBar = kXch + 4096;
+  // split-KV partials (after the last MMA): O_t f32 [128 rows][128 cols] of
+  // query tile t at kPart + t * 64 KB (over the Q and K areas), 16-byte chunks
+  // of a row permuted by chunk ^ (row & 7); (m, l) per row at kStats
+  static constexpr uint32_t kPart = kQ;
+  static constexpr uint32_t kStats = kXch + 4096;  // [2 tiles][128 rows] float2
+  static constexpr uint32_t kBar = kStats + 2048;
   static constexpr uint32_t kBytes = kBar + 256 + 1024;
 };
 
@@ -122,6 +144,83 @@ __device__ __forceinline__ float half_row_exp_store(const HalfRowS& s, uint32_t 
   return (sa + sb) + (sc + sd);
 }
 
+// Merge of query rows over the S partials of its cluster (split-KV): a warp
+// takes kRows rows at once, lane l owning output columns [4l, 4l + 4) of
+// each; every distributed-shared-memory load of the group is issued before
+// the first one is used, so the remote latency is paid once per group.
+template <int kRows, int kMaxS>
+__device__ __forceinline__ void merge_rows(const AttnFwdParams& p, uint8_t* smem, int S, const int (&R)[kRows],
+                                           int nrows, int b, int h, int qp, int lane) {
+  float ms[kRows][kMaxS], ls[kRows][kMaxS];
+  float4 os[kRows][kMaxS];
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) {
+    if (i >= nrows) break;
+    const int t = R[i] >> 7, row = R[i] & 127;
+    const uint32_t stats = smem_u32(smem + AttnSmem::kStats) + static_cast<uint32_t>(t * 128 + row) * 8u;
+    const int chunk = (lane & ~7) | ((lane & 7) ^ (row & 7));
+    const uint32_t part = smem_u32(smem + AttnSmem::kPart) + static_cast<uint32_t>(t) * 65536u +
+                          static_cast<uint32_t>(row) * 512u + static_cast<uint32_t>(chunk) * 16u;
+#pragma unroll
+    for (int s = 0; s < kMaxS; ++s) {
+      if (s < S) {
+        const float2 st = ld_cluster_f2(map_to_rank(stats, s));
+        os[i][s] = ld_cluster_f4(map_to_rank(part, s));
+        ms[i][s] = st.x;
+        ls[i][s] = st.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) {
+    if (i >= nrows) break;
+    const int qrow = qp * 256 + R[i];
+    float m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxS; ++s)
+      if (s < S) m = fmaxf(m, ms[i][s]);
+    float l = 0.f, o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxS; ++s) {
+      if (s < S) {
+        const float w = ex2_approx(ms[i][s] - m);
+        l = fmaf(ls[i][s], w, l);
+        o0 = fmaf(os[i][s].x, w, o0);
+        o1 = fmaf(os[i][s].y, w, o1);
+        o2 = fmaf(os[i][s].z, w, o2);
+        o3 = fmaf(os[i][s].w, w, o3);
+      }
+    }
+    if (qrow >= p.N) continue;
+    const float inv_l = 1.0f / l;
+    uint2 wv;
+    wv.x = pack_half2(o0 * inv_l, o1 * inv_l);
+    wv.y = pack_half2(o2 * inv_l, o3 * inv_l);
+    __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128 + lane * 4;
+    *reinterpret_cast<uint2*>(dst) = wv;
+    if (p.lse && lane == 0)
+      p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = (m + __log2f(l)) * 0.69314718055994531f;
+  }
+}
+
+// This CTA's share of the cluster's merge: rows [r0, r1) of the 256, warp w
+// taking rows r0 + w, r0 + w + 18, ... in groups of kRows.
+template <int kRows, int kMaxS>
+__device__ __forceinline__ void merge_share(const AttnFwdParams& p, uint8_t* smem, int S, int r0, int r1, int b,
+                                            int h, int qp, int warp, int lane) {
+  constexpr int kWarps = kAttnThreads / 32;
+  for (int base = r0 + warp; base < r1; base += kRows * kWarps) {
+    int R[kRows];
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      R[i] = base + i * kWarps;
+      if (R[i] < r1) n = i + 1;
+    }
+    merge_rows<kRows, kMaxS>(p, smem, S, R, n, b, h, qp, lane);
+  }
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,7 +241,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = warp_id(), lane = lane_id();
+  const int S = p.splits;
   int bid = blockIdx.x;
+  const int split = bid % S;  // = rank in the cluster (clusters are S consecutive CTAs along x)
+  bid = p.unit0 + bid / S;
   const int qp = bid % p.q_pairs;
   bid /= p.q_pairs;
   const int h = bid % p.Hq;
@@ -175,6 +277,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   grid_dep_wait();  // inputs of this call (q^, K, V, prefix lengths) are final from here on
   const int L = p.plen[b] + p.N;
   const int T = (L + 127) >> 7;
+  // this CTA's key tiles [j0, j0 + Ts); the host guarantees S <= T, so Ts >= 1
+  const int j0 = split * T / S;
+  const int Ts = (split + 1) * T / S - j0;
   const WaitGuard wg{abort_flag, p.status};
 
   if (warp == 0) {
@@ -188,17 +293,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         tma_load_3d(sQ + t * T32, &p.q_map, q_full, 0, qp * 256 + t * 128, qz);
         tma_load_3d(sQ + t * T32 + 16384, &p.q_map, q_full, 64, qp * 256 + t * 128, qz);
       }
-      for (int j = 0; j < T; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+      for (int jj = 0; jj < Ts; ++jj) {
+        const int s = jj & 1;
+        const uint32_t ph = (jj >> 1) & 1;
+        const int key0 = (j0 + jj) * 128;
         mbar_wait(&k_empty[s], ph ^ 1u, wg);
         mbar_expect_tx(&k_full[s], T32);
-        tma_load_3d(sK + s * T32, &p.k_map, &k_full[s], 0, j * 128, kz);
-        tma_load_3d(sK + s * T32 + 16384, &p.k_map, &k_full[s], 64, j * 128, kz);
+        tma_load_3d(sK + s * T32, &p.k_map, &k_full[s], 0, key0, kz);
+        tma_load_3d(sK + s * T32 + 16384, &p.k_map, &k_full[s], 64, key0, kz);
         mbar_wait(&v_empty[s], ph ^ 1u, wg);
         mbar_expect_tx(&v_full[s], T32);
-        tma_load_3d(sV + s * T32, &p.v_map, &v_full[s], 0, j * 128, kz);
-        tma_load_3d(sV + s * T32 + 16384, &p.v_map, &v_full[s], 64, j * 128, kz);
+        tma_load_3d(sV + s * T32, &p.v_map, &v_full[s], 0, key0, kz);
+        tma_load_3d(sV + s * T32 + 16384, &p.v_map, &v_full[s], 64, key0, kz);
       }
     }
   } else if (warp == 1) {
@@ -206,20 +312,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       constexpr uint32_t idesc_qk = idesc_f16(128, 128, false, false, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(128, 128, false, false, false, true);
       const uint32_t q_addr[2] = {smem_u32(sQ), smem_u32(sQ + T32)};
-      auto issue_s = [&](int t, int j) {
-        const uint32_t k_addr = smem_u32(sK + (j & 1) * T32);
+      auto issue_s = [&](int t, int jj) {
+        const uint32_t k_addr = smem_u32(sK + (jj & 1) * T32);
         const uint32_t qa = t ? q_addr[1] : q_addr[0];
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ss(tmem + t * 128u, kmajor_desc(qa, kk, 16384), kmajor_desc(k_addr, kk, 16384), idesc_qk, kk > 0);
         umma_commit(&s_full[t]);
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t va = smem_u32(sV + (j & 1) * T32);
+      auto issue_pv = [&](int t, int jj) {
+        const uint32_t va = smem_u32(sV + (jj & 1) * T32);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tmem + 256u + t * 128u, tmem + t * 128u + kk * 8u, mnmajor_desc(va, kk, 16384), idesc_pv,
-                  (j | kk) != 0);
+                  (jj | kk) != 0);
         umma_commit(&o_done[t]);
       };
       mbar_wait(q_full, 0, wg);
@@ -228,25 +334,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       issue_s(0, 0);
       issue_s(1, 0);
       umma_commit(&k_empty[0]);
-      for (int j = 0; j < T; ++j) {
-        const int s = j & 1;
-        const bool more = j + 1 < T;
-        mbar_wait(&v_full[s], (j >> 1) & 1, wg);
-        mbar_wait(&p_full[0], j & 1, wg);
+      for (int jj = 0; jj < Ts; ++jj) {
+        const int s = jj & 1;
+        const bool more = jj + 1 < Ts;
+        mbar_wait(&v_full[s], (jj >> 1) & 1, wg);
+        mbar_wait(&p_full[0], jj & 1, wg);
         tc_fence_after();
-        issue_pv(0, j);
+        issue_pv(0, jj);
         if (more) {
-          mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, wg);
+          mbar_wait(&k_full[(jj + 1) & 1], ((jj + 1) >> 1) & 1, wg);
           tc_fence_after();
-          issue_s(0, j + 1);  // overwrites P_0 only after the P V MMA above (in-order issue)
+          issue_s(0, jj + 1);  // overwrites P_0 only after the P V MMA above (in-order issue)
         }
-        mbar_wait(&p_full[1], j & 1, wg);
+        mbar_wait(&p_full[1], jj & 1, wg);
         tc_fence_after();
-        issue_pv(1, j);
+        issue_pv(1, jj);
         umma_commit(&v_empty[s]);
         if (more) {
-          issue_s(1, j + 1);
-          umma_commit(&k_empty[(j + 1) & 1]);
+          issue_s(1, jj + 1);
+          umma_commit(&k_empty[(jj + 1) & 1]);
         }
       }
     }
@@ -262,15 +368,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     float* xch = reinterpret_cast<float*>(smem + AttnSmem::kXch) + t * 512;  // [2 buffers][2 halves][128]
     const int bar_id = 1 + t;
     float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's partial row sum
-    for (int j = 0; j < T; ++j) {
-      mbar_wait(&s_full[t], j & 1, wg);
+    for (int jj = 0; jj < Ts; ++jj) {
+      mbar_wait(&s_full[t], jj & 1, wg);
       tc_fence_after();
-      const int valid = L - j * 128;  // keys of this tile that exist (>= 1)
+      const int valid = L - (j0 + jj) * 128;  // keys of this tile that exist (>= 1)
       const bool full = valid >= 128;
       HalfRowS srow;
       load_half_row(tS + col0, srow);
       const float pm = full ? half_row_max<true>(srow, col0, valid) : half_row_max<false>(srow, col0, valid);
-      float* xb = xch + (j & 1) * 256;
+      float* xb = xch + (jj & 1) * 256;
       xb[half * 128 + row] = pm;
       // both halves hold their scores in registers past this barrier, so P
       // may overwrite S; the partial maxima are exchanged through smem
@@ -278,7 +384,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const float m_tile = fmaxf(pm, xb[(half ^ 1) * 128 + row]) * p.scale_log2;
       bool need = false;
       float m_new = m_run;
-      if (j == 0) {
+      if (jj == 0) {
         m_new = m_tile;
       } else if (m_tile > m_run + kLazyRescaleLog2) {
         need = true;
@@ -287,8 +393,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // o_done completes once per P V of this tile; waiting on every phase in
       // order keeps the parity unambiguous. S_t of this tile was issued after
       // the previous P V, so that P V is already complete here: O is stable.
-      if (j >= 1) {
-        mbar_wait(&o_done[t], (j - 1) & 1, wg);
+      if (jj >= 1) {
+        mbar_wait(&o_done[t], (jj - 1) & 1, wg);
         tc_fence_after();
       }
       const float m_old = m_run;
@@ -314,36 +420,74 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
-    // epilogue: l = sum of the two halves; o = O / l for this half's 64 columns
-    mbar_wait(&o_done[t], (T - 1) & 1, wg);
+    // epilogue: l = sum of the two halves
+    mbar_wait(&o_done[t], (Ts - 1) & 1, wg);
     tc_fence_after();
-    float* xb = xch + (T & 1) * 256;
+    float* xb = xch + (Ts & 1) * 256;
     xb[half * 128 + row] = l_run;
     named_bar_sync(bar_id, 256);
     const float l_row = l_run + xb[(half ^ 1) * 128 + row];
-    const int qrow = qp * 256 + t * 128 + row;
-    const float inv_l = 1.0f / l_row;
-    __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128 + col0;
+    if (S == 1) {
+      // o = O / l for this half's 64 columns
+      const int qrow = qp * 256 + t * 128 + row;
+      const float inv_l = 1.0f / l_row;
+      __half* dst = p.out + (static_cast<long long>(b) * p.N + qrow) * (p.Hq * 128) + h * 128 + col0;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tO + col0 + c * 32, r);
-      tmem_ld_wait();
-      if (qrow < p.N) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + col0 + c * 32, r);
+        tmem_ld_wait();
+        if (qrow < p.N) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 w;
-          w.x = pack_half2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
-          w.y = pack_half2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
-          w.z = pack_half2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
-          w.w = pack_half2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
-          d4[i] = w;
+          for (int i = 0; i < 4; ++i) {
+            uint4 w;
+            w.x = pack_half2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
+            w.y = pack_half2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
+            w.z = pack_half2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
+            w.w = pack_half2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
+            d4[i] = w;
+          }
         }
       }
+      if (p.lse && half == 0 && qrow < p.N)
+        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = (m_run + __log2f(l_row)) * 0.69314718055994531f;
+    } else {
+      // split-KV partial: unnormalised O (this half's 64 columns) into this
+      // CTA's shared memory; the last MMA of the CTA is complete (every MMA
+      // reading Q or K was issued before the final P V of either tile)
+      float* part = reinterpret_cast<float*>(smem + AttnSmem::kPart + t * 65536) + row * 128;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + col0 + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int chunk = half * 16 + c * 8 + i;
+          const int phys = (chunk & ~7) | ((chunk & 7) ^ (row & 7));
+          *reinterpret_cast<uint4*>(part + phys * 4) =
+              make_uint4(r[4 * i + 0], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+        }
+      }
+      if (half == 0)
+        reinterpret_cast<float2*>(smem + AttnSmem::kStats)[t * 128 + row] = make_float2(m_run, l_row);
     }
-    if (p.lse && half == 0 && qrow < p.N)
-      p.lse[(static_cast<long long>(b) * p.Hq + h) * p.N + qrow] = (m_run + __log2f(l_row)) * 0.69314718055994531f;
+  }
+  if (S > 1) {
+    // every CTA of the cluster has its partial in shared memory
+    __syncwarp();
+    cluster_sync();
+    const int r0 = split * 256 / S, r1 = (split + 1) * 256 / S;
+    if (S == 2)
+      merge_share<4, 2>(p, smem, S, r0, r1, b, h, qp, warp, lane);
+    else if (S <= 4)
+      merge_share<2, 4>(p, smem, S, r0, r1, b, h, qp, warp, lane);
+    else
+      merge_share<1, kMaxAttnSplits>(p, smem, S, r0, r1, b, h, qp, warp, lane);
+    // no CTA leaves (releasing its shared memory) before all reads are done
+    __syncwarp();
+    cluster_sync();
   }
   tc_fence_before();
   __syncthreads();

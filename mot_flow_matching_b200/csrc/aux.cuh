@@ -16,25 +16,61 @@ struct PlenArray {
 // (bf16 -> f16, exact for |x| <= 65504 apart from f16 subnormals), rows
 // [plen[b] + N, Lcap) are zeroed so masked key tiles never hold NaN/Inf.
 // "Setup notes" (LoRA trainer docs): the prefix-KV cache is static input.
-// One thread moves 8 elements (16 bytes).
+// Only the rows this kernel owns are walked: Lcap - N per (branch, KV head),
+// row r < plen[b] maps to r, the rest to r + N. One thread moves 8 elements
+// (16 bytes). The same launch first converts the jobs in `cvt` (the f16
+// copies of the LoRA tensors that meet f16 operands, per call since a
+// trainer may update them in place), so a forward makes one launch for both.
+struct CvtJobs {
+  const __nv_bfloat16* src[6];
+  __half* dst[6];
+  long long n8[6];  // element count / 8
+  int count;
+};
+
+__device__ __forceinline__ bool cvt_jobs_run(const CvtJobs& jobs) {
+  bool overflow = false;
+  for (int j = 0; j < jobs.count; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(jobs.src[j]);
+    uint4* dst = reinterpret_cast<uint4*>(jobs.dst[j]);
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < jobs.n8[j];
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+      const uint4 r = src[i];
+      const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&r);
+      float2 f[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[k] = __bfloat1622float2(bv[k]);
+        overflow |= fabsf(f[k].x) > 65504.f || fabsf(f[k].y) > 65504.f;
+      }
+      dst[i] = make_uint4(pack_half2(f[0].x, f[0].y), pack_half2(f[1].x, f[1].y), pack_half2(f[2].x, f[2].y),
+                          pack_half2(f[3].x, f[3].y));
+    }
+  }
+  return overflow;
+}
+
 __global__ void __launch_bounds__(256) build_kv_kernel(const __nv_bfloat16* __restrict__ kc,
                                                        const __nv_bfloat16* __restrict__ vc,
                                                        __half* __restrict__ kall, __half* __restrict__ vall,
                                                        int Hkv, int Pmax, int N, int Lcap, long long total_chunks,
-                                                       PlenArray plen, int* status) {
+                                                       PlenArray plen, const CvtJobs cvt, int* status) {
   grid_dep_launch();
   grid_dep_wait();
-  bool overflow = false;
+  bool overflow = cvt_jobs_run(cvt);
+  const int own = Lcap - N;  // rows of one (branch, KV head) written here
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total_chunks;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int chunk = static_cast<int>(idx & 15);
-    const long long rowg = idx >> 4;
-    const int row = static_cast<int>(rowg % Lcap);
-    const long long bg = rowg / Lcap;
+    const long long rg = idx >> 4;
+    const int r = static_cast<int>(rg % own);
+    const long long bg = rg / own;
     const int b = static_cast<int>(bg / Hkv);
     const int pl = plen.v[b];
-    uint4* kd = reinterpret_cast<uint4*>(kall + rowg * 128 + chunk * 8);
-    uint4* vd = reinterpret_cast<uint4*>(vall + rowg * 128 + chunk * 8);
+    const int row = r < pl ? r : r + N;
+    const long long dst = (bg * Lcap + row) * 128 + chunk * 8;
+    uint4* kd = reinterpret_cast<uint4*>(kall + dst);
+    uint4* vd = reinterpret_cast<uint4*>(vall + dst);
     if (row < pl) {
       const long long src = (bg * Pmax + row) * 128 + chunk * 8;
       const uint4 kr = *reinterpret_cast<const uint4*>(kc + src);
@@ -54,7 +90,7 @@ __global__ void __launch_bounds__(256) build_kv_kernel(const __nv_bfloat16* __re
       }
       *kd = ko;
       *vd = vo;
-    } else if (row >= pl + N) {
+    } else {
       *kd = make_uint4(0, 0, 0, 0);
       *vd = make_uint4(0, 0, 0, 0);
     }
@@ -121,34 +157,55 @@ __global__ void __launch_bounds__(256) transpose_copy_kernel(const __nv_bfloat16
   }
 }
 
-// Several bf16 -> f16 conversions in one launch (LoRA tensors that meet f16
-// activations in an MMA; they may change between calls, so this runs per call).
-struct CvtJobs {
-  const __nv_bfloat16* src[6];
-  __half* dst[6];
-  long long n8[6];  // element count / 8
-  int count;
-};
-
+// bf16 -> f16 copies (tensors that meet f16 operands in an MMA), outside a forward
 __global__ void __launch_bounds__(256) cvt_multi_kernel(const CvtJobs jobs, int* status) {
   grid_dep_launch();
   grid_dep_wait();
-  bool overflow = false;
-  for (int j = 0; j < jobs.count; ++j) {
-    const uint4* src = reinterpret_cast<const uint4*>(jobs.src[j]);
-    uint4* dst = reinterpret_cast<uint4*>(jobs.dst[j]);
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < jobs.n8[j];
+  const bool overflow = cvt_jobs_run(jobs);
+  if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
+}
+
+// Zero-padded f16 copies of lora_up tensors: dst [rows, ld] holds src
+// [rows, r] (bf16) in columns [col0, col0 + r) and zeros elsewhere (col0, r
+// and ld multiples of 8). The gate and up LoRA-up tensors of the SwiGLU MLP
+// become the two blocks of a block-diagonal K extension this way: the gate
+// copy in columns [0, r) and the up copy in [RP, RP + r) of [I, 2 RP] rows,
+// against u = [s x A_gate^T | s x A_up^T].
+struct PadJobs {
+  const __nv_bfloat16* src[2];
+  __half* dst[2];
+  long long rows[2];
+  int r, ld, col0[2];
+  int count;
+};
+
+// Per-call preparation of the MLP's LoRA tensors in one launch: the plain
+// conversions in `cvt`, then the padded copies in `pad`.
+__global__ void __launch_bounds__(256) mlp_prep_kernel(const CvtJobs cvt, const PadJobs pad, int* status) {
+  grid_dep_launch();
+  grid_dep_wait();
+  bool overflow = cvt_jobs_run(cvt);
+  const int chunks_per_row = pad.ld / 8;
+  for (int j = 0; j < pad.count; ++j) {
+    const long long n = pad.rows[j] * chunks_per_row;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
-      const uint4 r = src[i];
-      const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&r);
-      float2 f[4];
+      const long long row = i / chunks_per_row;
+      const int col = static_cast<int>(i - row * chunks_per_row) * 8;
+      uint4 o = make_uint4(0, 0, 0, 0);
+      if (col >= pad.col0[j] && col < pad.col0[j] + pad.r) {
+        const uint4 v = *reinterpret_cast<const uint4*>(pad.src[j] + row * pad.r + (col - pad.col0[j]));
+        const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&v);
+        float2 f[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        f[k] = __bfloat1622float2(bv[k]);
-        overflow |= fabsf(f[k].x) > 65504.f || fabsf(f[k].y) > 65504.f;
+        for (int k = 0; k < 4; ++k) {
+          f[k] = __bfloat1622float2(bv[k]);
+          overflow |= fabsf(f[k].x) > 65504.f || fabsf(f[k].y) > 65504.f;
+        }
+        o = make_uint4(pack_half2(f[0].x, f[0].y), pack_half2(f[1].x, f[1].y), pack_half2(f[2].x, f[2].y),
+                       pack_half2(f[3].x, f[3].y));
       }
-      dst[i] = make_uint4(pack_half2(f[0].x, f[0].y), pack_half2(f[1].x, f[1].y), pack_half2(f[2].x, f[2].y),
-                          pack_half2(f[3].x, f[3].y));
+      *reinterpret_cast<uint4*>(pad.dst[j] + row * pad.ld + col) = o;
     }
   }
   if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);

@@ -72,6 +72,11 @@ struct GemmCore {
   // writes its f32 partial tile to split_ws; the CTA that finishes a tile
   // last (per-tile counter in split_cnt, which it resets) sums the partials
   // in split order into TMEM and runs the epilogue.
+  // pair kernel: the B rows of CTA rank r come from b_map[r] of every
+  // segment at rows [tn * BN/2, tn * BN/2 + BN/2) (regions unused), so one
+  // 256-column tile holds BN/2 columns of two different weights for the same
+  // output indices (the gate and up halves of a SwiGLU projection)
+  int b_by_rank;
   int k_splits;  // 1 = off
   int total_kb;  // host side: the smallest K-block total of any tile (bounds the split count)
   float4* split_ws;  // [tiles * k_splits][BN / 4][128]
@@ -464,7 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int si = 0; si < g.num_segs; ++si) {
       tma_prefetch_desc(&g.maps[g.segs[si].a_map]);
-      for (int r = 0; r < g.num_regions; ++r) tma_prefetch_desc(&g.maps[g.segs[si].b_map[r]]);
+      for (int r = 0; r < (g.b_by_rank ? 2 : g.num_regions); ++r) tma_prefetch_desc(&g.maps[g.segs[si].b_map[r]]);
     }
   }
   if (warp == 1) {
@@ -505,9 +510,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const int n = n0 + (i < nbox ? i : 0) * box_n;
-            const int r = region_of(g, n);
-            bmap[i] = &g.maps[sg.b_map[r]];
-            bcoord[i] = n - g.region_n0[r];
+            if (g.b_by_rank) {
+              bmap[i] = &g.maps[sg.b_map[rank]];
+              bcoord[i] = tn * kHalfN + (i < nbox ? i : 0) * box_n;
+            } else {
+              const int r = region_of(g, n);
+              bmap[i] = &g.maps[sg.b_map[r]];
+              bcoord[i] = n - g.region_n0[r];
+            }
           }
           const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
           for (int kb = 0; kb < nkb; ++kb) {
@@ -1060,6 +1070,148 @@ struct EpiQkv {
       }
 #pragma unroll
       for (int i = 0; i < 128; ++i) overflow |= fabsf(v[i]) > 65504.f;
+    }
+    if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
+  }
+};
+
+// SwiGLU epilogue of the gate/up projection (pair kernel with b_by_rank,
+// BN = 256): D columns [0, 128) of the tile are the gate pre-activation g and
+// [128, 256) the up pre-activation u of the same 128 intermediate indices
+// j0 = n0 / 2 + [0, 128). Stores h = silu(g) u as f16 [M, I] and, for
+// training, g and u themselves (f16, the backward's inputs). silu(g) =
+// g / (1 + 2^(-g log2 e)) with the MUFU exponential and reciprocal; the
+// exponent is capped so that 1 + e stays finite (silu -> 0 for g -> -inf).
+// "SenseNova-U1" (vLLM-Omni recipe), measured kernel table: act_and_mul
+// between the gate/up projection and down_proj, folded in here.
+struct EpiSwiGLU {
+  struct Params {
+    __half* h;       // [M, I]
+    __half* g_out;   // [M, I] or null
+    __half* u_out;   // [M, I] or null
+    int M, I;
+  };
+  __device__ __forceinline__ static float silu(float g) {
+    const float e = ex2_approx(fminf(-g * 1.4426950408889634f, 126.0f));
+    return g * __frcp_rn(1.0f + e);
+  }
+  template <int BN>
+  __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
+                                               int* status) {
+    static_assert(BN == 256, "128 gate + 128 up columns per tile");
+    const int m = m0 + row;
+    const int j0 = n0 >> 1;
+    bool overflow = false;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_ld32(taddr + c, gr);
+      tmem_ld32(taddr + 128 + c, ur);
+      tmem_ld_wait();
+      if (m >= p.M || j0 + c >= p.I) continue;
+      const long long off = static_cast<long long>(m) * p.I + j0 + c;
+      uint32_t hw[16];
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float g0 = __uint_as_float(gr[2 * k]), g1 = __uint_as_float(gr[2 * k + 1]);
+        const float u0 = __uint_as_float(ur[2 * k]), u1 = __uint_as_float(ur[2 * k + 1]);
+        const float h0 = silu(g0) * u0, h1 = silu(g1) * u1;
+        amax = fmax3_nan(amax, fabsf(h0), fabsf(h1));
+        hw[k] = pack_half2(h0, h1);
+      }
+      uint4* hd = reinterpret_cast<uint4*>(p.h + off);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) hd[q] = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+      if (p.g_out) {
+        uint4* gd = reinterpret_cast<uint4*>(p.g_out + off);
+        uint4* ud = reinterpret_cast<uint4*>(p.u_out + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t gw[4], uw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = 8 * q + 2 * k;
+            amax = fmax3_nan(amax, fabsf(__uint_as_float(gr[e])), fabsf(__uint_as_float(gr[e + 1])));
+            amax = fmax3_nan(amax, fabsf(__uint_as_float(ur[e])), fabsf(__uint_as_float(ur[e + 1])));
+            gw[k] = pack_half2(__uint_as_float(gr[e]), __uint_as_float(gr[e + 1]));
+            uw[k] = pack_half2(__uint_as_float(ur[e]), __uint_as_float(ur[e + 1]));
+          }
+          gd[q] = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+          ud[q] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+        }
+      }
+      overflow |= !(amax <= 65504.f);
+    }
+    if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
+  }
+};
+
+// SwiGLU backward epilogue of dh = dy W_down + s g_d A_down (pair kernel,
+// BN = 256 columns of I): with the forward's g, u (f16) at the same (m, j),
+//   dg = dh u silu'(g),  du = dh silu(g),
+//   silu'(g) = sigma(g) (1 + g (1 - sigma(g))),  sigma(g) = 1 / (1 + e^-g),
+// stored as f16 into one [M, 2I] tensor (dg in columns [0, I), du in
+// [I, 2I)), which the dx GEMM and the LoRA-gradient GEMMs read.
+struct EpiSwiGLUBwd {
+  struct Params {
+    __half* dgu;        // [M, 2I]
+    const __half* g;    // [M, I]
+    const __half* u;    // [M, I]
+    int M, I;
+  };
+  template <int BN>
+  __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
+                                               int* status) {
+    const int m = m0 + row;
+    bool overflow = false;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      const int j = n0 + c;
+      if (j >= p.I) break;  // the same for every thread
+      uint32_t dr[32];
+      tmem_ld32(taddr + c, dr);
+      tmem_ld_wait();
+      if (m >= p.M) continue;
+      const long long off = static_cast<long long>(m) * p.I + j;
+      const uint4* g4 = reinterpret_cast<const uint4*>(p.g + off);
+      const uint4* u4 = reinterpret_cast<const uint4*>(p.u + off);
+      uint4 gv[4], uv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gv[q] = g4[q];
+        uv[q] = u4[q];
+      }
+      uint32_t dgw[16], duw[16];
+      float amax = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __half2* gh = reinterpret_cast<const __half2*>(&gv[q]);
+        const __half2* uh = reinterpret_cast<const __half2*>(&uv[q]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 gf = __half22float2(gh[k]);
+          const float2 uf = __half22float2(uh[k]);
+          const float d0 = __uint_as_float(dr[8 * q + 2 * k]), d1 = __uint_as_float(dr[8 * q + 2 * k + 1]);
+          const float s0 = __frcp_rn(1.0f + ex2_approx(fminf(-gf.x * 1.4426950408889634f, 126.0f)));
+          const float s1 = __frcp_rn(1.0f + ex2_approx(fminf(-gf.y * 1.4426950408889634f, 126.0f)));
+          const float dg0 = d0 * uf.x * (s0 * (1.0f + gf.x * (1.0f - s0)));
+          const float dg1 = d1 * uf.y * (s1 * (1.0f + gf.y * (1.0f - s1)));
+          const float du0 = d0 * gf.x * s0, du1 = d1 * gf.y * s1;
+          amax = fmax3_nan(amax, fabsf(dg0), fabsf(dg1));
+          amax = fmax3_nan(amax, fabsf(du0), fabsf(du1));
+          dgw[4 * q + k] = pack_half2(dg0, dg1);
+          duw[4 * q + k] = pack_half2(du0, du1);
+        }
+      }
+      uint4* gd = reinterpret_cast<uint4*>(p.dgu + static_cast<long long>(m) * 2 * p.I + j);
+      uint4* ud = reinterpret_cast<uint4*>(p.dgu + static_cast<long long>(m) * 2 * p.I + p.I + j);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gd[q] = make_uint4(dgw[4 * q], dgw[4 * q + 1], dgw[4 * q + 2], dgw[4 * q + 3]);
+        ud[q] = make_uint4(duw[4 * q], duw[4 * q + 1], duw[4 * q + 2], duw[4 * q + 3]);
+      }
+      overflow |= !(amax <= 65504.f);
     }
     if (overflow) atomicOr(status, DEV_ERR_NUMERIC);
   }

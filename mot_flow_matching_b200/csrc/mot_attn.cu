@@ -1,8 +1,8 @@
 // mot_attn.cu -- C ABI of the gen-tower attention layer (see include/mot_attn.h).
 //
 // Forward launch sequence on the caller's stream (r = LoRA rank, s = alpha/r):
-//   [r>0] A_o -> f16 (it meets the f16 attention output in an MMA)
-//   build_kv      prefix rows of the f16 key/value buffers, zero tail rows
+//   build_kv      prefix rows of the f16 key/value buffers, zero tail rows;
+//                 [r>0] A_o and lora_up -> f16 (they meet f16 operands)
 //   [r>0] lora-down GEMM    u_qkv = s x [A_q; A_k; A_v]^T           (bf16)
 //   QKV GEMM + epilogue     x W_qkv^T + u B^T -> RMSNorm -> RoPE -> q^, K, V
 //   attention               o = softmax(q^ K^T / sqrt(dh)) V         (f16)
@@ -236,6 +236,95 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// launch_pdl for a kernel whose CTAs form clusters of `cluster` CTAs along x
+// (grid.x a multiple of it); cluster 1 is a plain launch
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               int cluster, const Args&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// Split-KV plan of the attention forward: how many clusters of S CTAs
+// (split-KV ranges) fit on the GPU at once, per S (index 1 = plain CTAs,
+// one per SM), queried once per handle from the occupancy calculator.
+void attn_cluster_caps(int (&cap)[kMaxAttnSplits + 1], int num_sms) {
+  set_smem_attr(attn_fwd_kernel, AttnSmem::kBytes);
+  cap[0] = 0;
+  cap[1] = num_sms;
+  for (int S = 2; S <= kMaxAttnSplits; ++S) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(S * 64);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = AttnSmem::kBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_fwd_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cap[S] = n;
+  }
+}
+
+// Split-KV plan of one attention forward. Units (b, h, query pair) run as
+// one CTA each in waves of cap[1] (one CTA per SM); when the last wave is
+// partly empty, the units of that tail may instead run as clusters of S
+// CTAs, each taking 1/S of the keys, merged through distributed shared
+// memory (a second launch, after the full waves). Cost in key steps (one
+// 128-key tile for both query tiles of a CTA, ~2.2 us on B200): per CTA a
+// fixed prologue/epilogue (kAttnFixedSteps) plus its key tiles, plus the
+// merge for split CTAs (kAttnMergeSteps); per launch, waves of cap[S]
+// clusters. Both constants come from timing forced split counts on the
+// 512^2, 1024^2 and 2048^2 workloads (a split of every unit never paid off
+// there: the fixed cost per CTA outweighs the balance it buys).
+constexpr double kAttnFixedSteps = 2.2, kAttnMergeSteps = 1.5;
+
+struct AttnPlan {
+  int full_units;  // units [0, full_units) unsplit
+  int splits;      // the rest as clusters of `splits` CTAs (1: none)
+};
+
+AttnPlan plan_attention(const int (&cap)[kMaxAttnSplits + 1], int units, int t_min, int t_max) {
+  const double step_full = t_max + kAttnFixedSteps;
+  const int waves = (units + cap[1] - 1) / cap[1];
+  AttnPlan best{units, 1};
+  double best_cost = waves * step_full;
+  const int full = (units / cap[1]) * cap[1];
+  const int tail = units - full;
+  if (tail == 0) return best;
+  for (int S = 2; S <= kMaxAttnSplits && S <= t_min; ++S) {
+    if (cap[S] <= 0) continue;
+    const double tail_waves = static_cast<double>((tail + cap[S] - 1) / cap[S]);
+    const double per_cta = static_cast<double>((t_max + S - 1) / S) + kAttnFixedSteps + kAttnMergeSteps;
+    const double cost = (full / cap[1]) * step_full + tail_waves * per_cta;
+    if (cost < best_cost - 1e-9) {
+      best = {full, S};
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 // let launch_gemm split K (1-CTA kernel; partials in ws of cap bytes, counters in cnt)
 void enable_split(GemmCore& c, void* ws, int* cnt, size_t cap = kSplitWsBytes) {
   c.k_splits = -1;
@@ -412,8 +501,15 @@ struct mot_attn {
   int* split_cnt = nullptr;  // [3][kSplitCounters] split-K arrival counters: backward (caller's / side stream), forward
   void* fsplit = nullptr;    // forward split-K partials (LoRA down), sized for max_batch x max_img_tokens
   size_t fsplit_bytes = 0;
+  int device = 0;  // the CUDA device the handle was created on
   int num_sms = 148;
   int last_launches = 0;
+  // attention split-KV: clusters of S CTAs resident at once, per S; a forced
+  // split count (0 = planned per call) and the count the last forward used
+  int attn_cap[kMaxAttnSplits + 1] = {};
+  int attn_splits_forced = 0;
+  int last_attn_splits = 0;
+  int last_attn_full_units = 0;
   // backward: a second stream for the gradient GEMMs nothing later depends on
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
@@ -515,10 +611,12 @@ void release(mot_attn* h) {
   delete h;
 }
 
-// launch bookkeeping shared by forward and backward: error capture, launch
-// count and the optional per-launch events
-struct Launches {
-  mot_attn* h;
+// launch bookkeeping shared by forward and backward (of the attention and
+// of the MLP handle): error capture, launch count and the optional
+// per-launch events
+template <class H>
+struct LaunchesT {
+  H* h;
   cudaStream_t st;   // the caller's stream
   cudaStream_t cur;  // where the next launch goes: st, or the handle's side stream
   int count = 0;
@@ -527,11 +625,11 @@ struct Launches {
   bool side_pending = false;  // side-stream work not yet joined into st
   cudaEvent_t last[2] = {};   // latest profiling event on st / on the side stream
   cudaError_t err = cudaSuccess;
-  Launches(mot_attn* handle, cudaStream_t s) : h(handle), st(s), cur(s) {
+  LaunchesT(H* handle, cudaStream_t s) : h(handle), st(s), cur(s) {
     if (h->profile) last[0] = mark(st);
   }
   // every return path leaves st ordered after the side stream's work
-  ~Launches() {
+  ~LaunchesT() {
     if (side_pending) join();
   }
   void note(cudaError_t e) {
@@ -576,6 +674,7 @@ struct Launches {
     return err == cudaSuccess ? MOT_OK : MOT_ERR_CUDA;
   }
 };
+using Launches = LaunchesT<mot_attn>;
 
 }  // namespace
 
@@ -646,6 +745,7 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
   h->RP = h->rank ? static_cast<int>(round_up(h->rank, 64)) : 0;
   int dev = 0;
   cudaGetDevice(&dev);
+  h->device = dev;
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -687,6 +787,7 @@ mot_status mot_attn_create(const mot_attn_config* cfg, const mot_attn_weights* w
   ok = ok && cudaGetLastError() == cudaSuccess && refresh_f16_copies(h, s) == cudaSuccess &&
        cudaStreamSynchronize(s) == cudaSuccess;
   if (ok) ok = build_weight_maps(h) == MOT_OK;
+  if (ok) attn_cluster_caps(h->attn_cap, h->num_sms);
   if (!ok) {
     release(h);
     return MOT_ERR_CUDA;
@@ -727,8 +828,11 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
   if (B > c.max_batch || N > c.max_img_tokens || P > c.max_prefix) return MOT_ERR_UNSUPPORTED_SHAPE;
   if (P > 0 && (!k_cache || !v_cache)) return MOT_ERR_INVALID_ARGUMENT;
-  for (int b = 0; b < B; ++b)
+  for (int b = 0; b < B; ++b) {
     if (prefix_len[b] < 0 || prefix_len[b] > P) return MOT_ERR_INVALID_ARGUMENT;
+    // a forced split-KV count needs at least one key tile per split in every branch
+    if (h->attn_splits_forced > (prefix_len[b] + N + 127) / 128) return MOT_ERR_UNSUPPORTED_SHAPE;
+  }
   const void* ptrs[] = {x, y, y_f32, saved, workspace, k_cache, v_cache};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return MOT_ERR_ALIGNMENT;
@@ -759,36 +863,37 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   const int qd = Hq * 128, kvd = Hkv * 128, nqkv = qd + 2 * kvd;
   Launches lz(h, st);
 
-  // 1. f16 copies of A_o and of every lora_up (they meet f16 operands); per
-  //    call, since a trainer updates them in place between calls
+  // 1. one launch: the f16 copies of A_o and of every lora_up (they meet f16
+  //    operands; per call, since a trainer updates them in place between
+  //    calls) and the key/value buffers' prefix rows (cache -> f16) and zero
+  //    tail rows
   const int outj[3] = {qd, kvd, kvd};
-  lz.stage = ST_CVT_LORA_O;
-  if (r > 0) {
-    CvtJobs jobs{};
-    const void* src[5] = {h->w.a_o, h->w.b_o, h->w.b_q, h->w.b_k, h->w.b_v};
-    __half* dst[5] = {ao16, bo16, bqkv16, bqkv16 + static_cast<long long>(qd) * r,
-                      bqkv16 + static_cast<long long>(qd + kvd) * r};
-    const long long n[5] = {static_cast<long long>(r) * qd, static_cast<long long>(d) * r,
-                            static_cast<long long>(qd) * r, static_cast<long long>(kvd) * r,
-                            static_cast<long long>(kvd) * r};
-    for (int i = 0; i < 5; ++i) {
-      jobs.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
-      jobs.dst[i] = dst[i];
-      jobs.n8[i] = n[i] / 8;
-    }
-    jobs.count = 5;
-    lz.done(launch_pdl(cvt_multi_kernel, dim3(2 * h->num_sms), dim3(256), 0, st, jobs, h->status));
-  }
-  // 2. key/value buffers: prefix rows + zero tail
   lz.stage = ST_BUILD_KV;
   {
+    CvtJobs jobs{};
+    if (r > 0) {
+      const void* src[5] = {h->w.a_o, h->w.b_o, h->w.b_q, h->w.b_k, h->w.b_v};
+      __half* dst[5] = {ao16, bo16, bqkv16, bqkv16 + static_cast<long long>(qd) * r,
+                        bqkv16 + static_cast<long long>(qd + kvd) * r};
+      const long long n[5] = {static_cast<long long>(r) * qd, static_cast<long long>(d) * r,
+                              static_cast<long long>(qd) * r, static_cast<long long>(kvd) * r,
+                              static_cast<long long>(kvd) * r};
+      for (int i = 0; i < 5; ++i) {
+        jobs.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
+        jobs.dst[i] = dst[i];
+        jobs.n8[i] = n[i] / 8;
+      }
+      jobs.count = 5;
+    }
     PlenArray pl{};
     for (int b = 0; b < B; ++b) pl.v[b] = prefix_len[b];
-    const long long chunks = static_cast<long long>(B) * Hkv * L.Lcap * 16;
-    const int grid = static_cast<int>(std::min<long long>((chunks + 255) / 256, 16LL * h->num_sms));
+    // rows [0, plen) and [plen + N, Lcap) of every (branch, KV head), 16 chunks each
+    const long long chunks = static_cast<long long>(B) * Hkv * (L.Lcap - N) * 16;
+    const long long want = std::max<long long>((chunks + 255) / 256, r > 0 ? 2LL * h->num_sms : 1LL);
+    const int grid = static_cast<int>(std::min<long long>(want, 16LL * h->num_sms));
     lz.done(launch_pdl(build_kv_kernel, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(k_cache),
                        static_cast<const __nv_bfloat16*>(v_cache), k_all, v_all, Hkv, std::max(P, 1), N, L.Lcap,
-                       chunks, pl, h->status));
+                       chunks, pl, jobs, h->status));
   }
   // 3. LoRA down for q/k/v: u_qkv[:, j*RP:(j+1)*RP] = s x A_j^T (f16)
   lz.stage = ST_LORA_DOWN_QKV;
@@ -876,14 +981,34 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ap.Hkv = Hkv;
     ap.Lcap = L.Lcap;
     ap.q_pairs = (N + 255) / 256;
-    for (int b = 0; b < B; ++b) ap.plen[b] = prefix_len[b];
+    int t_min = 1 << 30, t_max = 0;
+    for (int b = 0; b < B; ++b) {
+      ap.plen[b] = prefix_len[b];
+      const int T = (prefix_len[b] + N + 127) / 128;
+      t_min = std::min(t_min, T);
+      t_max = std::max(t_max, T);
+    }
+    const int units = B * Hq * ap.q_pairs;
+    const AttnPlan plan = h->attn_splits_forced > 0 ? AttnPlan{0, h->attn_splits_forced}
+                                                    : plan_attention(h->attn_cap, units, t_min, t_max);
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
     ap.out = attn;
     ap.lse = lse;
     ap.status = h->status;
-    static std::once_flag once;
-    std::call_once(once, [] { set_smem_attr(attn_fwd_kernel, AttnSmem::kBytes); });
-    lz.done(launch_pdl(attn_fwd_kernel, dim3(B * Hq * ap.q_pairs), dim3(kAttnThreads), AttnSmem::kBytes, st, ap));
+    h->last_attn_splits = plan.full_units < units ? plan.splits : 1;
+    h->last_attn_full_units = plan.full_units;
+    if (plan.full_units > 0) {
+      ap.splits = 1;
+      ap.unit0 = 0;
+      lz.done(launch_pdl_cluster(attn_fwd_kernel, dim3(plan.full_units), dim3(kAttnThreads), AttnSmem::kBytes, st,
+                                 1, ap));
+    }
+    if (plan.full_units < units) {
+      ap.splits = plan.splits;
+      ap.unit0 = plan.full_units;
+      lz.done(launch_pdl_cluster(attn_fwd_kernel, dim3((units - plan.full_units) * plan.splits), dim3(kAttnThreads),
+                                 AttnSmem::kBytes, st, plan.splits, ap));
+    }
   }
   // 6. LoRA down for o: u_o = s o A_o^T (f16; training also keeps it as a bf16 hi + lo pair)
   lz.stage = ST_LORA_DOWN_O;
@@ -1411,10 +1536,16 @@ extern "C" mot_status mot_attn_forward_noalloc(mot_attn_t h, const void* x, int3
                                                void* stream) {
   if (!h || !x || !y || !prefix_len) return MOT_ERR_INVALID_ARGUMENT;
   if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
-  size_t need = 0;
-  const mot_status st = mot_attn_query_sizes(&h->cfg, B, N, P, &need, nullptr);
-  if (st != MOT_OK) return st;
-  if (need > kNoAllocScratchBytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
+  const mot_attn_config& c = h->cfg;
+  if (B > c.max_batch || N > c.max_img_tokens || P > c.max_prefix) return MOT_ERR_UNSUPPORTED_SHAPE;
+  // the scratch array is resolved for the current device: it must be the
+  // handle's, where its weights and copies live
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return MOT_ERR_CUDA;
+  if (cur != h->device) return MOT_ERR_INVALID_ARGUMENT;
+  // what an inference forward of this shape needs (what mot_attn_forward checks)
+  const Layout L = make_layout(c, B, N, P, false);
+  if (L.fwd_scratch + L.act_bytes > kNoAllocScratchBytes) return MOT_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = noalloc_scratch_address();
   if (!scratch) return MOT_ERR_CUDA;
   return mot_attn_forward(h, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, nullptr, 0, scratch,
@@ -1550,6 +1681,17 @@ mot_status mot_dev_stage_timeline(mot_attn_t h, int32_t* ids, float* t0_ms, floa
   return MOT_OK;
 }
 
+mot_status mot_dev_set_attn_splits(mot_attn_t h, int32_t splits) {
+  if (!h || splits < 0 || splits > kMaxAttnSplits) return MOT_ERR_INVALID_ARGUMENT;
+  if (splits > 1 && h->attn_cap[splits] <= 0) return MOT_ERR_UNSUPPORTED_SHAPE;
+  h->attn_splits_forced = splits;
+  return MOT_OK;
+}
+
+int32_t mot_dev_last_attn_splits(mot_attn_t h) { return h ? h->last_attn_splits : 0; }
+
+int32_t mot_dev_last_attn_full_units(mot_attn_t h) { return h ? h->last_attn_full_units : 0; }
+
 mot_status mot_dev_wait_probe(mot_attn_t h, void* stream) {
   if (!h) return MOT_ERR_INVALID_ARGUMENT;
   wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->status);
@@ -1574,3 +1716,6 @@ mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ the gen-tower MLP
+#include "mot_mlp.cuh"

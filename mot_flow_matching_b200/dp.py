@@ -13,7 +13,9 @@ initialised (NCCL on GPUs, gloo in the CPU tests).
 """
 import datetime
 import os
-from typing import Mapping, Optional, Tuple
+import socket
+import subprocess
+from typing import Mapping, Optional, Sequence, Tuple
 
 
 def world_info(env: Optional[Mapping[str, str]] = None) -> Tuple[int, int, int]:
@@ -70,3 +72,48 @@ def finish(world: int) -> None:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+
+
+def free_port() -> int:
+    """A TCP port on 127.0.0.1 that nothing listens on right now."""
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def check_world(requested: int, env: Optional[Mapping[str, str]] = None) -> str:
+    """How a command asked for `requested` ranks (one per GPU) should run:
+    "run" when it is already one of the launcher's ranks and the launcher's
+    world size is the request (or one rank was asked for without a
+    launcher), "spawn" when no launcher started it and it must start the
+    ranks itself. A launcher world size that differs from the request is an
+    error (the job would report a GPU count it did not use)."""
+    env = os.environ if env is None else env
+    if requested < 1:
+        raise ValueError(f"rank count must be >= 1, got {requested}")
+    if "WORLD_SIZE" not in env:
+        return "spawn" if requested > 1 else "run"
+    world, _, _ = world_info(env)
+    if world != requested:
+        raise ValueError(f"launched with WORLD_SIZE={world} but {requested} ranks were requested")
+    return "run"
+
+
+def spawn_local_ranks(nprocs: int, argv: Sequence[str], master_port: Optional[int] = None,
+                      extra_env: Optional[Mapping[str, str]] = None) -> int:
+    """Run `argv` as ranks 0..nprocs-1 of one job on this node (rank i on
+    local GPU i), the way a launcher would: each child gets RANK, LOCAL_RANK,
+    WORLD_SIZE and a MASTER_ADDR/MASTER_PORT on 127.0.0.1, inherits stdout
+    and stderr, and is waited for. Returns the first non-zero exit code (0
+    when every rank succeeded)."""
+    port = master_port or free_port()
+    procs = []
+    for rank in range(nprocs):
+        env = dict(os.environ)
+        env.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(nprocs),
+                    "LOCAL_WORLD_SIZE": str(nprocs), "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+        if extra_env:
+            env.update(extra_env)
+        procs.append(subprocess.Popen(list(argv), env=env))
+    codes = [p.wait() for p in procs]
+    return next((c for c in codes if c != 0), 0)

@@ -169,6 +169,19 @@ def mot_dev_wait_probe(h, stream=None) -> None:
     check(lib().mot_dev_wait_probe(h, _stream(stream)), "mot_dev_wait_probe")
 
 
+def mot_dev_set_attn_splits(h, splits: int) -> None:
+    """0: split-KV count planned per call; 1..8: forced (tests, measurements)."""
+    check(lib().mot_dev_set_attn_splits(h, int(splits)), "mot_dev_set_attn_splits")
+
+
+def mot_dev_last_attn_splits(h) -> int:
+    return int(lib().mot_dev_last_attn_splits(h))
+
+
+def mot_dev_last_attn_full_units(h) -> int:
+    return int(lib().mot_dev_last_attn_full_units(h))
+
+
 def mot_dev_profile(h, enable: bool) -> None:
     check(lib().mot_dev_profile(h, int(bool(enable))), "mot_dev_profile")
 

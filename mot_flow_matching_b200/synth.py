@@ -164,6 +164,37 @@ def make_mlp_inputs(tokens: int, hidden: int, inter: int, lora_rank: int, seed_b
     return out
 
 
+# MLP workloads: the same calls as the attention workloads (tokens = all CFG
+# branches' image tokens), intermediate width 12288 (3 x hidden; the pages
+# give no dense width), the same LoRA ranks
+MLP_INTER = 3 * HIDDEN
+
+
+@dataclasses.dataclass(frozen=True)
+class MlpWorkload:
+    name: str
+    tokens: int
+    lora_rank: int
+    lora_alpha: float
+    train: bool = False
+    hidden: int = HIDDEN
+    inter: int = MLP_INTER
+
+
+MLP_WORKLOADS = {
+    0: MlpWorkload("mlp_512sq_b1", 256, 16, 16.0),
+    1: MlpWorkload("mlp_1024sq_cfg2", 2048, 32, 32.0),
+    2: MlpWorkload("mlp_2048sq_cfg2", 8192, 32, 32.0),
+    4: MlpWorkload("mlp_train_2048sq_b1", 4096, 32, 32.0, train=True),
+}
+
+
+def mlp_workload_inputs(index: int, with_dy: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+    wl = MLP_WORKLOADS[index]
+    return make_mlp_inputs(wl.tokens, wl.hidden, wl.inter, wl.lora_rank, 1000 * index,
+                           wl.train if with_dy is None else with_dy)
+
+
 def workload_inputs(index: int, with_dy: Optional[bool] = None, shard: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(WORKLOADS[index], 1000 * index, with_dy, shard)
 

@@ -84,3 +84,41 @@ def test_shards_share_weights_and_split_data():
         assert not torch.equal(s0[k], s1[k]), k
     for k in ("w_q", "w_k", "w_v", "w_o", "q_norm", "k_norm", "a_q", "b_o"):
         assert torch.equal(s0[k], s1[k]), k
+
+
+def _bench(args, env_extra=None, timeout=240):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, env=env, capture_output=True,
+                          text=True, timeout=timeout)
+
+
+def test_bench_gpus_two_spawns_two_ranks():
+    # no launcher: bench.py --gpus 2 starts two ranks itself (gloo on CPU here)
+    res = _bench(["--gpus", "2", "--steps", "3", "--check-ranks"])
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(l) for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["local_rank"] == 0
+    s0, s1 = line["shard_sums"]
+    assert s0 != s1  # each rank ran its own data shard
+    assert line["value"] > 0
+
+
+def test_bench_rejects_a_launcher_world_size_that_differs():
+    res = _bench(["--gpus", "2", "--steps", "3", "--check-ranks"],
+                 {"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
+    assert res.returncode == 2
+    assert "WORLD_SIZE=1" in res.stderr
+
+
+def test_check_world():
+    assert dp.check_world(1, {}) == "run"
+    assert dp.check_world(4, {}) == "spawn"
+    assert dp.check_world(2, {"WORLD_SIZE": "2", "RANK": "1"}) == "run"
+    with pytest.raises(ValueError):
+        dp.check_world(8, {"WORLD_SIZE": "1", "RANK": "0"})
