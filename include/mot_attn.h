@@ -140,6 +140,31 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t batch, int32_t 
                             int32_t prefix_max, void* y, float* y_f32, void* saved, size_t saved_bytes,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* The prefix tower's attention layer over the prompt, which builds the
+ * prefix-KV cache entry of this layer ("SenseNova-U1" DiffSynth-Studio docs,
+ * architecture note: the prompt is encoded once by the understanding branch
+ * into past_key_values; "Setup notes", "Why bf16 base on CPU + tower
+ * offload?": the prefix tower computes the static cache once, in bf16). The
+ * handle is created with that tower's weights (w_q .. w_o, q_norm, k_norm of
+ * the *_mot modules; lora_rank 0 for the pages' setup, adapters are applied
+ * if the handle has them). Per branch b, token i < lengths[b] at position i:
+ *   q, k, v as mot_attn_forward; o_i = softmax over keys j <= i; y = o Wo^T;
+ *   k_cache_out[b, g, i] = k^_i (normalised, rotated), v_cache_out[b, g, i] = v_i
+ * so that k_cache_out / v_cache_out with prefix_len = lengths are exactly the
+ * cache mot_attn_forward takes (the image tokens continue at position
+ * lengths[b]).
+ *   x           device bf16 [B, N, d]     prompt hidden states (N = padded length)
+ *   lengths     host int32 [B], 1 <= lengths[b] <= N; rows at or beyond it
+ *               are padding: their y and cache rows are unspecified
+ *   y, y_f32    as mot_attn_forward (y_f32 may be NULL)
+ *   k_cache_out, v_cache_out  device bf16 [B, Hkv, N, dh], each element one
+ *               round to nearest of the f32 value
+ *   workspace   device, workspace_bytes of mot_attn_query_sizes(cfg, B, N, 0)
+ * 1 <= B <= max_batch, N <= max_img_tokens. Inference only. */
+mot_status mot_attn_prefix_forward(mot_attn_t h, const void* x, int32_t batch, int32_t tokens,
+                                   const int32_t* lengths, void* y, float* y_f32, void* k_cache_out,
+                                   void* v_cache_out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* LoRA-training backward of the layer (base weights, norm gains and the
  * cache are frozen; no gradient flows into them).
  *   dy       device bf16 [B, N, d]     upstream gradient of y

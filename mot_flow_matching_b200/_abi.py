@@ -57,6 +57,8 @@ SIGNATURES = {
     "mot_attn_backward": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                     POINTER(c_int32), c_int32, c_void_p, c_size_t, c_void_p, c_void_p,
                                     POINTER(c_void_p), POINTER(c_void_p), c_int32, c_void_p, c_size_t, c_void_p]),
+    "mot_attn_prefix_forward": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, POINTER(c_int32), c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "mot_attn_forward_noalloc": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p,
                                            POINTER(c_int32), c_int32, c_void_p, c_void_p, c_void_p]),
     "mot_attn_query_host_staging": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32,

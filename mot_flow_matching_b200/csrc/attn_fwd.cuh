@@ -56,6 +56,10 @@ struct AttnFwdParams {
   int B, N, Hq, Hkv, Lcap, q_pairs;  // q_pairs = ceil(N / 256)
   int splits;                        // S: key-range splits = cluster size (1..kMaxAttnSplits)
   int unit0;                         // first (b, h, query pair) unit of this launch
+  // causal (prefix tower): plen[b] is the branch's token count L_b (keys and
+  // queries are the same N-row sequence); query i attends to keys j <= i,
+  // j < L_b. Otherwise keys are [cache ; self], L_b = plen[b] + N.
+  int causal;
   int plen[kMaxBatch];
   float scale_log2;  // log2(e) / sqrt(dh)
   __half* out;       // [B*N, Hq*dh] token-major
@@ -275,8 +279,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   const uint32_t tmem = *tmem_slot;
   grid_dep_launch();
   grid_dep_wait();  // inputs of this call (q^, K, V, prefix lengths) are final from here on
-  const int L = p.plen[b] + p.N;
-  const int T = (L + 127) >> 7;
+  const int L = p.causal ? p.plen[b] : p.plen[b] + p.N;
+  // causal: no key past the unit's last query row is needed
+  const int T = ((p.causal ? min(L, qp * 256 + 256) : L) + 127) >> 7;
   // this CTA's key tiles [j0, j0 + Ts); the host guarantees S <= T, so Ts >= 1
   const int j0 = split * T / S;
   const int Ts = (split + 1) * T / S - j0;
@@ -368,10 +373,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     float* xch = reinterpret_cast<float*>(smem + AttnSmem::kXch) + t * 512;  // [2 buffers][2 halves][128]
     const int bar_id = 1 + t;
     float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's partial row sum
+    // keys this row may see: all L, or (causal) those up to its own position
+    const int key_end = p.causal ? min(L, qp * 256 + t * 128 + row + 1) : L;
     for (int jj = 0; jj < Ts; ++jj) {
       mbar_wait(&s_full[t], jj & 1, wg);
       tc_fence_after();
-      const int valid = L - (j0 + jj) * 128;  // keys of this tile that exist (>= 1)
+      const int valid = key_end - (j0 + jj) * 128;  // keys of this tile this row sees (>= 1 on the first tile)
       const bool full = valid >= 128;
       HalfRowS srow;
       load_half_row(tS + col0, srow);

@@ -996,6 +996,12 @@ struct EpiQkv {
     const float* gamma_q;
     const float* gamma_k;
     const float2* rope;  // [positions][64] (cos, sin)
+    // prefix tower: the layer's cache entry, bf16 [B, Hkv, Pc, dh] keys
+    // (normalised, rotated) and values at row n, rounded once from f32; null
+    // for the gen tower
+    __nv_bfloat16* kc_out;
+    __nv_bfloat16* vc_out;
+    int Pc;
     int plen[kMaxBatch];
     int N, Hq, Hkv, Lcap, M;
     float eps;
@@ -1067,6 +1073,16 @@ struct EpiQkv {
         w.z = pack_half2(v[8 * i + 4], v[8 * i + 5]);
         w.w = pack_half2(v[8 * i + 6], v[8 * i + 7]);
         d4[i] = w;
+      }
+      if (p.kc_out && head >= p.Hq) {
+        const bool is_k = head < p.Hq + p.Hkv;
+        const int g = head - p.Hq - (is_k ? 0 : p.Hkv);
+        uint4* c4 = reinterpret_cast<uint4*>((is_k ? p.kc_out : p.vc_out) +
+                                             (static_cast<long long>(b * p.Hkv + g) * p.Pc + n) * 128);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          c4[i] = make_uint4(pack_bf162(v[8 * i + 0], v[8 * i + 1]), pack_bf162(v[8 * i + 2], v[8 * i + 3]),
+                             pack_bf162(v[8 * i + 4], v[8 * i + 5]), pack_bf162(v[8 * i + 6], v[8 * i + 7]));
       }
 #pragma unroll
       for (int i = 0; i < 128; ++i) overflow |= fabsf(v[i]) > 65504.f;

@@ -819,10 +819,23 @@ mot_status mot_attn_get_device_status(mot_attn_t h, void* stream) {
   return MOT_OK;
 }
 
-mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, const void* k_cache,
-                            const void* v_cache, const int32_t* prefix_len, int32_t P, void* y, float* y_f32,
-                            void* saved, size_t saved_bytes, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The prefix tower's call (mot_attn_prefix_forward): the call's N tokens are
+// the prompt itself, at positions 0..N-1, attending causally to each other
+// (lengths[b] real tokens in branch b); the layer's cache entry (normalised,
+// rotated keys and values) is written as bf16 [B, Hkv, N, dh].
+struct PrefixCall {
+  const int32_t* lengths;
+  void* k_out;
+  void* v_out;
+};
+
+mot_status forward_impl(mot_attn_t h, const void* x, int32_t B, int32_t N, const void* k_cache, const void* v_cache,
+                        const int32_t* prefix_len, int32_t P, void* y, float* y_f32, void* saved, size_t saved_bytes,
+                        void* workspace, size_t workspace_bytes, void* stream, const PrefixCall* pc) {
   if (!h || !x || !y || !prefix_len || !workspace) return MOT_ERR_INVALID_ARGUMENT;
   const mot_attn_config& c = h->cfg;
   if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
@@ -831,7 +844,7 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
   for (int b = 0; b < B; ++b) {
     if (prefix_len[b] < 0 || prefix_len[b] > P) return MOT_ERR_INVALID_ARGUMENT;
     // a forced split-KV count needs at least one key tile per split in every branch
-    if (h->attn_splits_forced > (prefix_len[b] + N + 127) / 128) return MOT_ERR_UNSUPPORTED_SHAPE;
+    if (!pc && h->attn_splits_forced > (prefix_len[b] + N + 127) / 128) return MOT_ERR_UNSUPPORTED_SHAPE;
   }
   const void* ptrs[] = {x, y, y_f32, saved, workspace, k_cache, v_cache};
   for (const void* p : ptrs)
@@ -965,6 +978,11 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ep.Lcap = L.Lcap;
     ep.M = M;
     ep.eps = c.rms_eps;
+    if (pc) {
+      ep.kc_out = static_cast<__nv_bfloat16*>(pc->k_out);
+      ep.vc_out = static_cast<__nv_bfloat16*>(pc->v_out);
+      ep.Pc = N;
+    }
     lz.done(launch_gemm2<256, 6, EpiQkv>(core, ep, h->num_sms, st));
   }
   // 5. attention
@@ -983,14 +1001,17 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     ap.q_pairs = (N + 255) / 256;
     int t_min = 1 << 30, t_max = 0;
     for (int b = 0; b < B; ++b) {
-      ap.plen[b] = prefix_len[b];
+      ap.plen[b] = pc ? pc->lengths[b] : prefix_len[b];
       const int T = (prefix_len[b] + N + 127) / 128;
       t_min = std::min(t_min, T);
       t_max = std::max(t_max, T);
     }
+    ap.causal = pc ? 1 : 0;
     const int units = B * Hq * ap.q_pairs;
-    const AttnPlan plan = h->attn_splits_forced > 0 ? AttnPlan{0, h->attn_splits_forced}
-                                                    : plan_attention(h->attn_cap, units, t_min, t_max);
+    // causal units have unequal key ranges: they run unsplit
+    const AttnPlan plan = pc ? AttnPlan{units, 1}
+                          : h->attn_splits_forced > 0 ? AttnPlan{0, h->attn_splits_forced}
+                                                      : plan_attention(h->attn_cap, units, t_min, t_max);
     ap.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
     ap.out = attn;
     ap.lse = lse;
@@ -1053,6 +1074,32 @@ mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, c
     lz.done(launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   return lz.finish();
+}
+
+}  // namespace
+
+extern "C" {
+
+mot_status mot_attn_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, const void* k_cache,
+                            const void* v_cache, const int32_t* prefix_len, int32_t P, void* y, float* y_f32,
+                            void* saved, size_t saved_bytes, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return forward_impl(h, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, saved, saved_bytes, workspace,
+                      workspace_bytes, stream, nullptr);
+}
+
+mot_status mot_attn_prefix_forward(mot_attn_t h, const void* x, int32_t B, int32_t N, const int32_t* lengths,
+                                   void* y, float* y_f32, void* k_cache_out, void* v_cache_out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!h || !lengths || !k_cache_out || !v_cache_out) return MOT_ERR_INVALID_ARGUMENT;
+  if (B <= 0 || B > kMaxBatch || N <= 0) return MOT_ERR_INVALID_ARGUMENT;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 1 || lengths[b] > N) return MOT_ERR_INVALID_ARGUMENT;
+  if (!aligned16(k_cache_out) || !aligned16(v_cache_out)) return MOT_ERR_ALIGNMENT;
+  int32_t zeros[kMaxBatch] = {};
+  const PrefixCall pc{lengths, k_cache_out, v_cache_out};
+  return forward_impl(h, x, B, N, nullptr, nullptr, zeros, 0, y, y_f32, nullptr, 0, workspace, workspace_bytes,
+                      stream, &pc);
 }
 
 mot_status mot_attn_backward(mot_attn_t h, const void* dy, const void* x, int32_t B, int32_t N, const void* k_cache,

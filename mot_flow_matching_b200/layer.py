@@ -63,6 +63,17 @@ def mot_attn_forward(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequ
                                  _stream(stream)), "mot_attn_forward")
 
 
+def mot_attn_prefix_forward(h, x, batch, tokens, lengths: Sequence[int], y, k_cache_out, v_cache_out, y_f32=None,
+                            workspace=None, stream=None) -> None:
+    """The prefix tower's layer over the prompt (causal), writing the layer's
+    bf16 cache entry; see include/mot_attn.h."""
+    ln = (c_int32 * batch)(*[int(v) for v in lengths])
+    check(lib().mot_attn_prefix_forward(h, _ptr(x), batch, tokens, ln, _ptr(y), _ptr(y_f32), _ptr(k_cache_out),
+                                        _ptr(v_cache_out), _ptr(workspace),
+                                        workspace.numel() if workspace is not None else 0, _stream(stream)),
+          "mot_attn_prefix_forward")
+
+
 def mot_attn_forward_noalloc(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max,
                              y, y_f32=None, stream=None) -> None:
     """Forward whose scratch is the library's own fixed device array (no
@@ -241,6 +252,23 @@ class MotAttnLayer:
             workspace = self.workspace(B, N, P, x.device)
         mot_attn_forward(self.handle, x, B, N, k_cache, v_cache, prefix_len, P, y, y_f32, saved, workspace, stream)
         return y
+
+    def prefix_forward(self, x, lengths, y=None, y_f32=None, k_cache_out=None, v_cache_out=None, workspace=None,
+                       stream=None):
+        """Prefix-tower layer over the prompt x [B, N, d]: returns (y, k_cache, v_cache)."""
+        B, N, d = x.shape
+        c = self.cfg
+        if y is None:
+            y = torch.empty_like(x)
+        shape = (B, c.n_kv_heads, N, c.head_dim)
+        if k_cache_out is None:
+            k_cache_out = torch.empty(shape, dtype=torch.bfloat16, device=x.device)
+        if v_cache_out is None:
+            v_cache_out = torch.empty(shape, dtype=torch.bfloat16, device=x.device)
+        if workspace is None:
+            workspace = self.workspace(B, N, 0, x.device)
+        mot_attn_prefix_forward(self.handle, x, B, N, lengths, y, k_cache_out, v_cache_out, y_f32, workspace, stream)
+        return y, k_cache_out, v_cache_out
 
     def host_staging(self, batch, img_tokens, prefix_max, device="cuda"):
         n = mot_attn_query_host_staging(self.cfg, batch, img_tokens, prefix_max)

@@ -32,7 +32,7 @@ Readings where the pages give no formula:
      uncond): x0 = x0_u + img_cfg (x0_i - x0_u) + cfg (x0_c - x0_i); one
      branch: x0 = x0_c.
   S5 Euler on the straight flow z_s = (1 - s) x0 + s noise: velocity
-     v = (x0 - z) / max(sigma, t_eps), z <- z + (sigma_next - sigma) v
+     v = (z - x0) / max(sigma, t_eps), z <- z + (sigma_next - sigma) v
      (t_eps keeps the division away from sigma = 0).
   S6 shifted schedule: sigma_i = shift u_i / (1 + (shift - 1) u_i),
      u_i = 1 - i / steps, i = 0..steps.
@@ -76,7 +76,7 @@ def guidance(x0: np.ndarray, cfg: float, img_cfg: float) -> np.ndarray:
 
 def euler_update(z: np.ndarray, x0: np.ndarray, sigma: float, sigma_next: float, t_eps: float) -> np.ndarray:
     """One Euler step of S5."""
-    v = (x0 - z) / max(sigma, t_eps)
+    v = (z - x0) / max(sigma, t_eps)
     return z + (sigma_next - sigma) * v
 
 
