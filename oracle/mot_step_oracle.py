@@ -62,7 +62,7 @@ def timestep_embedding(sigma: float, dim: int) -> np.ndarray:
 def sigma_schedule(steps: int, shift: float) -> np.ndarray:
     """sigma_0 = 1 > ... > sigma_steps = 0 (S6)."""
     u = 1.0 - np.arange(steps + 1, dtype=np.float64) / steps
-    return u / (shift - (shift - 1.0) * u)
+    return shift * u / (1.0 + (shift - 1.0) * u)
 
 
 def guidance(x0: np.ndarray, cfg: float, img_cfg: float) -> np.ndarray:
