@@ -47,6 +47,15 @@ class MotMlpWeights(ctypes.Structure):
                                         "b_down")]
 
 
+class MotStepConfig(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("hidden", c_int32), ("patch_dim", c_int32), ("rms_eps", c_float)]
+
+
+class MotStepModel(ctypes.Structure):
+    _fields_ = [("attn", POINTER(c_void_p)), ("mlp", POINTER(c_void_p)), ("norm_in", POINTER(c_void_p)),
+                ("norm_post", POINTER(c_void_p)), ("w_in", c_void_p), ("norm_out", c_void_p), ("w_out", c_void_p)]
+
+
 # name -> (restype, argtypes); every symbol the headers declare
 SIGNATURES = {
     "mot_attn_query_sizes": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32, POINTER(c_size_t),
@@ -98,6 +107,12 @@ SIGNATURES = {
     "mot_dev_mlp_profile": (c_int32, [c_void_p, c_int32]),
     "mot_dev_mlp_stage_times": (c_int32, [c_void_p, POINTER(c_int32), POINTER(c_float), c_int32, POINTER(c_int32)]),
     "mot_dev_mlp_stage_name": (c_char_p, [c_int32]),
+    "mot_step_create": (c_int32, [POINTER(MotStepConfig), POINTER(MotStepModel), c_void_p, POINTER(c_void_p)]),
+    "mot_step_query_workspace": (c_int32, [c_void_p, c_int32, c_int32, c_int32, POINTER(c_size_t)]),
+    "mot_step_forward": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, POINTER(c_void_p), POINTER(c_void_p),
+                                   POINTER(c_int32), c_int32, c_float, c_float, c_float, c_float, c_float, c_void_p,
+                                   c_void_p, c_void_p, c_size_t, c_void_p]),
+    "mot_step_destroy": (None, [c_void_p]),
 }
 
 _lib = None

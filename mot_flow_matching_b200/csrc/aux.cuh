@@ -211,6 +211,104 @@ __global__ void __launch_bounds__(256) mlp_prep_kernel(const CvtJobs cvt, const 
   if (overflow && status) atomicOr(status, DEV_ERR_NUMERIC);
 }
 
+// ------------------------------------------------------------------ denoise step
+// RMSNorm of rows of the f32 residual stream into the bf16 input of the next
+// block: out[m] = RNE_bf16(h[m] / sqrt(mean(h[m]^2) + eps) * gain). With
+// `src` (the step's first norm) row m first becomes src[m % src_rows] + bias
+// (the patch embedding plus the timestep embedding, the same for every
+// branch) and is written back to h. One warp per row; d a multiple of 128.
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(float* __restrict__ h, const float* __restrict__ src,
+                                                           int src_rows, const float* __restrict__ bias,
+                                                           const float* __restrict__ gain,
+                                                           __nv_bfloat16* __restrict__ out, int rows, int d,
+                                                           float eps) {
+  grid_dep_launch();
+  grid_dep_wait();
+  const int lane = threadIdx.x & 31;
+  const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  for (int m = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); m < rows; m += nwarps) {
+    float* hr = h + static_cast<long long>(m) * d;
+    float ss = 0.f;
+    if (src) {
+      const float* sr = src + static_cast<long long>(m % src_rows) * d;
+      for (int c = lane * 4; c < d; c += 128) {
+        float4 v = *reinterpret_cast<const float4*>(sr + c);
+        const float4 b4 = *reinterpret_cast<const float4*>(bias + c);
+        v.x += b4.x;
+        v.y += b4.y;
+        v.z += b4.z;
+        v.w += b4.w;
+        *reinterpret_cast<float4*>(hr + c) = v;
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+    } else {
+      for (int c = lane * 4; c < d; c += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(hr + c);
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = rsqrtf(ss / static_cast<float>(d) + eps);
+    __nv_bfloat16* orow = out + static_cast<long long>(m) * d;
+    for (int c = lane * 4; c < d; c += 128) {
+      const float4 v = *reinterpret_cast<const float4*>(hr + c);
+      const float4 g = *reinterpret_cast<const float4*>(gain + c);
+      *reinterpret_cast<uint2*>(orow + c) =
+          make_uint2(pack_bf162(v.x * rs * g.x, v.y * rs * g.y), pack_bf162(v.z * rs * g.z, v.w * rs * g.w));
+    }
+  }
+}
+
+// Timestep embedding of the step (f32 [d]): cos(1000 sigma f_k) at k and
+// sin(1000 sigma f_k) at d/2 + k, f_k = 10000^(-k/(d/2)), in double.
+__global__ void temb_kernel(float* __restrict__ out, int d, double sigma) {
+  grid_dep_launch();
+  grid_dep_wait();
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < d / 2) {
+    const double ang = 1000.0 * sigma * pow(10000.0, -static_cast<double>(k) / (d / 2));
+    out[k] = static_cast<float>(cos(ang));
+    out[d / 2 + k] = static_cast<float>(sin(ang));
+  }
+}
+
+// Guidance over the branches' x0 predictions (cfg_norm none; branch order
+// cond, [image-cond,] uncond) and the Euler update of the image's patch
+// tokens: z_next = z + c (z - x0), c = (sigma_next - sigma) / max(sigma,
+// t_eps), also as bf16 for the next step's embedding GEMM. x0 [B, n], z [n].
+__global__ void __launch_bounds__(256) cfg_euler_kernel(const float* __restrict__ x0, long long n, int B,
+                                                        const float* __restrict__ z, float* __restrict__ z_next,
+                                                        __nv_bfloat16* __restrict__ z_next16, float cfg,
+                                                        float img_cfg, float c) {
+  grid_dep_launch();
+  grid_dep_wait();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float x;
+    if (B == 1)
+      x = x0[i];
+    else if (B == 2)
+      x = x0[n + i] + cfg * (x0[i] - x0[n + i]);
+    else
+      x = x0[2 * n + i] + img_cfg * (x0[n + i] - x0[2 * n + i]) + cfg * (x0[i] - x0[n + i]);
+    const float zi = z[i];
+    const float zn = zi + c * (zi - x);
+    z_next[i] = zn;
+    if (z_next16) z_next16[i] = __float2bfloat16_rn(zn);
+  }
+}
+
+// f32 -> bf16, round to nearest even (the patch tokens as a GEMM operand)
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ src,
+                                                          __nv_bfloat16* __restrict__ dst, long long n) {
+  grid_dep_launch();
+  grid_dep_wait();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
 // 2^x of a buffer through exp2_poly2 (accuracy tests of the softmax's FMA-pipe exponential)
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int npairs) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

@@ -833,10 +833,14 @@ struct PrefixCall {
   void* v_out;
 };
 
+// residual: the layer output is added into y_f32 (a residual stream the
+// caller keeps in f32; y may then be NULL) instead of overwriting y / y_f32
 mot_status forward_impl(mot_attn_t h, const void* x, int32_t B, int32_t N, const void* k_cache, const void* v_cache,
                         const int32_t* prefix_len, int32_t P, void* y, float* y_f32, void* saved, size_t saved_bytes,
-                        void* workspace, size_t workspace_bytes, void* stream, const PrefixCall* pc) {
-  if (!h || !x || !y || !prefix_len || !workspace) return MOT_ERR_INVALID_ARGUMENT;
+                        void* workspace, size_t workspace_bytes, void* stream, const PrefixCall* pc,
+                        bool residual = false) {
+  if (!h || !x || !prefix_len || !workspace) return MOT_ERR_INVALID_ARGUMENT;
+  if (residual ? !y_f32 : !y) return MOT_ERR_INVALID_ARGUMENT;
   const mot_attn_config& c = h->cfg;
   if (B <= 0 || N <= 0 || P < 0) return MOT_ERR_INVALID_ARGUMENT;
   if (B > c.max_batch || N > c.max_img_tokens || P > c.max_prefix) return MOT_ERR_UNSUPPORTED_SHAPE;
@@ -1068,9 +1072,10 @@ mot_status forward_impl(mot_attn_t h, const void* x, int32_t B, int32_t N, const
       core.num_segs = 2;
     }
     EpiStore::Params ep = store_params(M, d);
-    set_out16(ep, 0, y, d, true);
+    if (y) set_out16(ep, 0, y, d, true);
     ep.out32 = y_f32;
     ep.ld32 = d;
+    ep.accumulate32 = residual ? 1 : 0;
     lz.done(launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   return lz.finish();
@@ -1766,3 +1771,6 @@ mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32
 
 // ------------------------------------------------------------------ the gen-tower MLP
 #include "mot_mlp.cuh"
+
+// ------------------------------------------------------------------ the denoise step
+#include "mot_step.cuh"

@@ -279,9 +279,17 @@ mot_status mot_mlp_get_device_status(mot_mlp_t h, void* stream) {
   return MOT_OK;
 }
 
-mot_status mot_mlp_forward(mot_mlp_t h, const void* x, int32_t T, void* y, float* y_f32, void* saved,
-                           size_t saved_bytes, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!h || !x || !y || !workspace) return MOT_ERR_INVALID_ARGUMENT;
+}  // extern "C"
+
+namespace {
+
+// residual: the block output is added into y_f32 (the caller's f32
+// residual stream; y may then be NULL)
+mot_status mlp_forward_impl(mot_mlp_t h, const void* x, int32_t T, void* y, float* y_f32, void* saved,
+                            size_t saved_bytes, void* workspace, size_t workspace_bytes, void* stream,
+                            bool residual) {
+  if (!h || !x || !workspace) return MOT_ERR_INVALID_ARGUMENT;
+  if (residual ? !y_f32 : !y) return MOT_ERR_INVALID_ARGUMENT;
   const mot_mlp_config& c = h->cfg;
   if (T <= 0) return MOT_ERR_INVALID_ARGUMENT;
   if (T > c.max_tokens) return MOT_ERR_UNSUPPORTED_SHAPE;
@@ -416,12 +424,22 @@ mot_status mot_mlp_forward(mot_mlp_t h, const void* x, int32_t T, void* y, float
       core.num_segs = 2;
     }
     EpiStore::Params ep = store_params(T, d);
-    set_out16(ep, 0, y, d, true);
+    if (y) set_out16(ep, 0, y, d, true);
     ep.out32 = y_f32;
     ep.ld32 = d;
+    ep.accumulate32 = residual ? 1 : 0;
     lz.done(launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st));
   }
   return lz.finish();
+}
+
+}  // namespace
+
+extern "C" {
+
+mot_status mot_mlp_forward(mot_mlp_t h, const void* x, int32_t T, void* y, float* y_f32, void* saved,
+                           size_t saved_bytes, void* workspace, size_t workspace_bytes, void* stream) {
+  return mlp_forward_impl(h, x, T, y, y_f32, saved, saved_bytes, workspace, workspace_bytes, stream, false);
 }
 
 mot_status mot_mlp_backward(mot_mlp_t h, const void* dy, const void* x, int32_t T, const void* saved,

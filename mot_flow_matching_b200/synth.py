@@ -195,6 +195,35 @@ def mlp_workload_inputs(index: int, with_dy: Optional[bool] = None) -> Dict[str,
                            wl.train if with_dy is None else with_dy)
 
 
+# the denoise step's own tensors (patch embedding, norms, head) and the
+# noisy image; indices apart from the layers' tensors
+_STEP_TENSOR_INDEX = {"w_in": 60, "norm_out": 61, "w_out": 62, "z": 63, "norm_in": 64, "norm_post": 65}
+
+
+def make_step_inputs(n_layers: int, wl: Workload, inter: int, patch_dim: int, seed_base: int):
+    """CPU tensors for one denoise step over ``n_layers`` gen-tower layers:
+    per layer the attention layer's tensors (``make_inputs``, seed
+    seed_base + 100 l) with its prefix cache, the MLP's (``make_mlp_inputs``)
+    and the two norm gains (1 + 0.1 N(0, 1)); the tower's w_in [d, C] and
+    w_out [C, d] (N(0, 0.02)), norm_out; the image's patch tokens z [N, C]
+    (f32, N(0, 1))."""
+    d = wl.dims.hidden
+    s = lambda name, l=0: seed_base + _STEP_TENSOR_INDEX[name] + 100 * l
+    layers = []
+    for l in range(n_layers):
+        t = make_inputs(wl, seed_base + 100 * l, with_dy=False)
+        m = make_mlp_inputs(wl.batch * wl.img_tokens, d, inter, wl.lora_rank, seed_base + 100 * l + 50)
+        t.update({"mlp_" + k: v for k, v in m.items() if k != "x"})
+        t["norm_in"] = _draw((d,), 0.1, 1.0, s("norm_in", l))
+        t["norm_post"] = _draw((d,), 0.1, 1.0, s("norm_post", l))
+        layers.append(t)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(s("z"))
+    return {"layers": layers, "w_in": _draw((d, patch_dim), 0.02, 0.0, s("w_in")),
+            "norm_out": _draw((d,), 0.1, 1.0, s("norm_out")), "w_out": _draw((patch_dim, d), 0.02, 0.0, s("w_out")),
+            "z": torch.randn(wl.img_tokens, patch_dim, generator=g, dtype=torch.float32)}
+
+
 def workload_inputs(index: int, with_dy: Optional[bool] = None, shard: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(WORKLOADS[index], 1000 * index, with_dy, shard)
 
