@@ -224,6 +224,37 @@ def make_step_inputs(n_layers: int, wl: Workload, inter: int, patch_dim: int, se
             "z": torch.randn(wl.img_tokens, patch_dim, generator=g, dtype=torch.float32)}
 
 
+# the A3B gen tower's mixture-of-experts MLP: hidden 2048, 32 experts, top-8,
+# expert width 768 ("SenseNova-U1" vLLM-Omni recipe, A3B variant)
+MOE_HIDDEN, MOE_EXPERTS, MOE_TOP_K, MOE_INTER = 2048, 32, 8, 768
+_MOE_TENSOR_INDEX = {"x": 80, "w_router": 81, "w_gate": 82, "w_up": 83, "w_down": 84}
+
+
+def make_moe_inputs(tokens: int, hidden: int, inter: int, experts: int, seed_base: int) -> Dict[str, torch.Tensor]:
+    """CPU bf16 tensors for one MoE MLP call: x [tokens, hidden] N(0, 1);
+    w_router [E, hidden], w_gate, w_up [E, inter, hidden], w_down [E, hidden,
+    inter], all N(0, 0.02) (the attention layer's weight recipe)."""
+    s = lambda name: seed_base + _MOE_TENSOR_INDEX[name]
+    return {"x": _draw((tokens, hidden), 1.0, 0.0, s("x")),
+            "w_router": _draw((experts, hidden), 0.02, 0.0, s("w_router")),
+            "w_gate": _draw((experts, inter, hidden), 0.02, 0.0, s("w_gate")),
+            "w_up": _draw((experts, inter, hidden), 0.02, 0.0, s("w_up")),
+            "w_down": _draw((experts, hidden, inter), 0.02, 0.0, s("w_down"))}
+
+
+def draw_device(shape, std: float, mean: float, seed: int, device) -> torch.Tensor:
+    """bf16 N(mean, std^2) drawn on the device from a seeded generator of that
+    device (the large multi-layer benchmark stacks; the oracle never sees these)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    t = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t.to(torch.bfloat16)
+
+
 def workload_inputs(index: int, with_dy: Optional[bool] = None, shard: int = 0) -> Dict[str, torch.Tensor]:
     return make_inputs(WORKLOADS[index], 1000 * index, with_dy, shard)
 
