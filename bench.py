@@ -464,6 +464,148 @@ def mlp_steps(dev, flush, stream, args, world):
     return out
 
 
+STEP_LAYERS = 42  # decoder layers of the gen tower ("SenseNova-U1" DiffSynth-Studio docs, architecture note)
+
+
+def denoise_step_bench(dev, flush, stream, args, world):
+    """One gen-tower denoise step over all 42 layers (attention + MLP, LoRA
+    rank 32 on both) for the 2048^2 CFG call (B = 2, N = 4096, P = 400),
+    weights drawn on the device per layer; plus the prefix-tower layer that
+    builds one layer's cache for two 400-token prompts. CUDA events, L2
+    flushed before every step."""
+    import torch
+    from mot_flow_matching_b200 import dp, synth
+    from mot_flow_matching_b200.layer import MotAttnLayer
+    from mot_flow_matching_b200.mlp import MotMlp
+    from mot_flow_matching_b200.step import MotStep
+    wl = synth.WORKLOADS[WORKLOAD_INDEX]
+    d, r, I, C = wl.dims.hidden, wl.lora_rank, synth.MLP_INTER, 3 * 32 * 32
+    qd, kvd = wl.dims.n_q_heads * wl.dims.head_dim, wl.dims.n_kv_heads * wl.dims.head_dim
+    B, N, P = wl.batch, wl.img_tokens, wl.prefix
+    draw = lambda shape, std, mean, seed: synth.draw_device(shape, std, mean, seed, dev)
+    attn, mlps, keep = [], [], []
+    for l in range(STEP_LAYERS):
+        sd = 900_000 + 100 * l
+        a = {"w_q": draw((qd, d), 0.02, 0.0, sd + 1), "w_k": draw((kvd, d), 0.02, 0.0, sd + 2),
+             "w_v": draw((kvd, d), 0.02, 0.0, sd + 3), "w_o": draw((d, qd), 0.02, 0.0, sd + 4),
+             "q_norm": draw((128,), 0.1, 1.0, sd + 5), "k_norm": draw((128,), 0.1, 1.0, sd + 6)}
+        for i, (n, shape) in enumerate({"a_q": (r, d), "a_k": (r, d), "a_v": (r, d), "a_o": (r, qd), "b_q": (qd, r),
+                                        "b_k": (kvd, r), "b_v": (kvd, r), "b_o": (d, r)}.items()):
+            a[n] = draw(shape, 1 / 16 if n.startswith("a_") else 0.01, 0.0, sd + 10 + i)
+        m = {"w_gate": draw((I, d), 0.02, 0.0, sd + 30), "w_up": draw((I, d), 0.02, 0.0, sd + 31),
+             "w_down": draw((d, I), 0.02, 0.0, sd + 32)}
+        for i, (n, shape) in enumerate({"a_gate": (r, d), "a_up": (r, d), "a_down": (r, I), "b_gate": (I, r),
+                                        "b_up": (I, r), "b_down": (d, r)}.items()):
+            m[n] = draw(shape, 1 / 16 if n.startswith("a_") else 0.01, 0.0, sd + 40 + i)
+        cache = (draw((B, wl.dims.n_kv_heads, P, 128), 1.0, 0.0, sd + 60),
+                 draw((B, wl.dims.n_kv_heads, P, 128), 1.0, 0.0, sd + 61))
+        norms = (draw((d,), 0.1, 1.0, sd + 70), draw((d,), 0.1, 1.0, sd + 71))
+        attn.append(MotAttnLayer(a, lora_rank=r, lora_alpha=wl.lora_alpha, max_batch=B, max_img_tokens=N,
+                                 max_prefix=P))
+        mlps.append(MotMlp(m, lora_rank=r, lora_alpha=wl.lora_alpha, max_tokens=B * N, intermediate=I))
+        keep.append((a, m, cache, norms))
+    w_in, norm_out, w_out = draw((d, C), 0.02, 0.0, 990_001), draw((d,), 0.1, 1.0, 990_002), draw((C, d), 0.02, 0.0,
+                                                                                                   990_003)
+    step = MotStep(attn, mlps, [k[3][0] for k in keep], [k[3][1] for k in keep], w_in, norm_out, w_out)
+    z = torch.randn(N, C, generator=torch.Generator(device=dev).manual_seed(990_004), device=dev)
+    zn = torch.empty_like(z)
+    kc, vc = [k[2][0] for k in keep], [k[2][1] for k in keep]
+    pl = [P] * B
+    ws = step.workspace(B, N, P, dev)
+    for _ in range(2):
+        step.forward(z, kc, vc, pl, 0.6, 0.55, z_next=zn, workspace=ws)
+    torch.cuda.synchronize(dev)
+    dp.barrier(world)
+    steps = 3
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step.forward(z, kc, vc, pl, 0.6, 0.55, z_next=zn, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    for a in attn:
+        assert a.device_status() == 0
+    for m in mlps:
+        assert m.device_status() == 0
+    t = dp.max_over_ranks(statistics.mean(ms), world, dev)
+    peaks, _ = load_peaks()
+    layer_fl = sum(stage_work(wl, n)[0] for n in ("lora_down_qkv", "qkv_gemm", "attn_fwd", "lora_down_o", "o_gemm"))
+    fl = STEP_LAYERS * (layer_fl + mlp_flops(synth.MLP_WORKLOADS[MLP_INDEX])) + 2.0 * N * C * d + 2.0 * B * N * C * d
+    out = {"workload": f"denoise_step_2048sq_cfg2_{STEP_LAYERS}layers", "layers": STEP_LAYERS, "batch": B,
+           "img_tokens": N, "prefix": P, "lora_rank": r, "ms_per_step": t, "image_tokens_per_s": world * B * N / (t / 1e3),
+           "tflops": fl / (t / 1e3) / 1e12, "frac_of_bf16_peak": fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "algorithmic_tflop": fl / 1e12}
+    step.close()
+    # the prefix-tower layer that builds a layer's cache: two 400-token prompts
+    a0 = keep[0][0]
+    base = {k: v for k, v in a0.items() if not k.startswith(("a_", "b_"))}
+    player = MotAttnLayer(base, max_batch=B, max_img_tokens=P, max_prefix=0)
+    xp = draw((B, P, d), 1.0, 0.0, 990_010)
+    for _ in range(3):
+        player.prefix_forward(xp, [P] * B)
+    torch.cuda.synchronize(dev)
+    pms = []
+    for _ in range(5):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        player.prefix_forward(xp, [P] * B)
+        e1.record(stream)
+        e1.synchronize()
+        pms.append(e0.elapsed_time(e1))
+    assert player.device_status() == 0
+    player.close()
+    pt = dp.max_over_ranks(statistics.mean(pms), world, dev)
+    pfl = 2.0 * B * P * d * (qd + 2 * kvd) + 2.0 * B * wl.dims.n_q_heads * P * (P + 1) * 128 + 2.0 * B * P * qd * d
+    out["prefix_layer"] = {"batch": B, "prompt_tokens": P, "ms": pt, "tflops": pfl / (pt / 1e3) / 1e12}
+    for a in attn:
+        a.close()
+    for m in mlps:
+        m.close()
+    return out
+
+
+def moe_bench(dev, flush, stream, args, world):
+    """The A3B gen tower's mixture-of-experts MLP (hidden 2048, 32 experts,
+    top 8, width 768) over the 8192 image tokens of a 2048^2 CFG call;
+    weights and tokens drawn on the device; CUDA events, L2 flushed."""
+    import torch
+    from mot_flow_matching_b200 import dp, synth
+    from mot_flow_matching_b200.moe import MotMoe
+    T, d, E, K, I = 8192, synth.MOE_HIDDEN, synth.MOE_EXPERTS, synth.MOE_TOP_K, synth.MOE_INTER
+    draw = lambda shape, std, seed: synth.draw_device(shape, std, 0.0, seed, dev)
+    w = {"w_router": draw((E, d), 0.02, 980_001), "w_gate": draw((E, I, d), 0.02, 980_002),
+         "w_up": draw((E, I, d), 0.02, 980_003), "w_down": draw((E, d, I), 0.02, 980_004)}
+    x = draw((T, d), 1.0, 980_005)
+    moe = MotMoe(w, top_k=K, max_tokens=T)
+    y = torch.empty_like(x)
+    ws = moe.workspace(T, dev)
+    for _ in range(args.warmup):
+        moe.forward(x, y=y, workspace=ws)
+    torch.cuda.synchronize(dev)
+    dp.barrier(world)
+    ms = []
+    for _ in range(max(3, args.steps // 2)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moe.forward(x, y=y, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    assert moe.device_status() == 0
+    moe.close()
+    t = dp.max_over_ranks(statistics.mean(ms), world, dev)
+    fl = 6.0 * T * K * d * I + 2.0 * T * d * E
+    peaks, _ = load_peaks()
+    return {"workload": "moe_a3b_2048sq_cfg2_tokens", "tokens": T, "hidden": d, "experts": E, "top_k": K,
+            "intermediate": I, "ms": t, "tokens_per_s": world * T / (t / 1e3), "tflops": fl / (t / 1e3) / 1e12,
+            "frac_of_bf16_peak": fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"]}
+
+
 def sustained_steps(bundle, dev, stream, args, world, local):
     """Back-to-back forwards of one workload for at least args.sustained_s
     seconds under one pair of CUDA events, SM clock sampled throughout;
@@ -706,6 +848,16 @@ def run_ours(args):
     if not args.skip_mlp:
         mlp = mlp_steps(dev, flush, stream, args, world)
 
+    # the A3B tower's mixture-of-experts MLP
+    moe = None
+    if not args.skip_mlp:
+        moe = moe_bench(dev, flush, stream, args, world)
+
+    # one full denoise step (42 layers) and the prefix-tower layer
+    denoise = None
+    if not args.skip_step:
+        denoise = denoise_step_bench(dev, flush, stream, args, world)
+
     # sustained: back-to-back 2048^2 CFG forwards for >= 2 s, clocks sampled
     sustained = None
     if args.sustained_s > 0:
@@ -763,6 +915,8 @@ def run_ours(args):
             "also": also,
             "train": train,
             "mlp": mlp,
+            "denoise_step": denoise,
+            "moe": moe,
             "sustained": sustained,
         }
         print(json.dumps(line), flush=True)
@@ -810,6 +964,7 @@ def main():
     ap.add_argument("--skip-also", action="store_true")
     ap.add_argument("--skip-train", action="store_true")
     ap.add_argument("--skip-mlp", action="store_true")
+    ap.add_argument("--skip-step", action="store_true", help="skip the 42-layer denoise step and the prefix layer")
     ap.add_argument("--sustained-s", type=float, default=2.0,
                     help="seconds of back-to-back forwards for the sustained figure (0: skip)")
     ap.add_argument("--cpu-rows", type=int, default=512)

@@ -56,6 +56,15 @@ class MotStepModel(ctypes.Structure):
                 ("norm_post", POINTER(c_void_p)), ("w_in", c_void_p), ("norm_out", c_void_p), ("w_out", c_void_p)]
 
 
+class MotMoeConfig(ctypes.Structure):
+    _fields_ = [("hidden", c_int32), ("intermediate", c_int32), ("experts", c_int32), ("top_k", c_int32),
+                ("max_tokens", c_int32)]
+
+
+class MotMoeWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("w_router", "w_gate", "w_up", "w_down")]
+
+
 # name -> (restype, argtypes); every symbol the headers declare
 SIGNATURES = {
     "mot_attn_query_sizes": (c_int32, [POINTER(MotAttnConfig), c_int32, c_int32, c_int32, POINTER(c_size_t),
@@ -113,6 +122,12 @@ SIGNATURES = {
                                    POINTER(c_int32), c_int32, c_float, c_float, c_float, c_float, c_float, c_void_p,
                                    c_void_p, c_void_p, c_size_t, c_void_p]),
     "mot_step_destroy": (None, [c_void_p]),
+    "mot_moe_query_workspace": (c_int32, [POINTER(MotMoeConfig), c_int32, POINTER(c_size_t)]),
+    "mot_moe_create": (c_int32, [POINTER(MotMoeConfig), POINTER(MotMoeWeights), c_void_p, POINTER(c_void_p)]),
+    "mot_moe_forward": (c_int32, [c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                  c_void_p]),
+    "mot_moe_get_device_status": (c_int32, [c_void_p, c_void_p]),
+    "mot_moe_destroy": (None, [c_void_p]),
 }
 
 _lib = None

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmotattn.so")
 SOURCES = ["mot_attn.cu"]
-HEADERS = ["ptx.cuh", "gemm.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "aux.cuh", "mot_mlp.cuh", "mot_step.cuh"]
+HEADERS = ["ptx.cuh", "gemm.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "aux.cuh", "mot_mlp.cuh", "mot_step.cuh", "moe.cuh", "mot_moe.cuh"]
 
 
 def nvcc_path() -> str:

@@ -77,6 +77,13 @@ struct GemmCore {
   // 256-column tile holds BN/2 columns of two different weights for the same
   // output indices (the gate and up halves of a SwiGLU projection)
   int b_by_rank;
+  // pair kernel, grouped GEMM (mixture of experts): M tile tm (256 rows)
+  // belongs to group tile_group[tm] (device memory, written by an earlier
+  // kernel; -1: an unused tile, skipped by every role), whose B rows start
+  // at tile_group[tm] * group_rows of each B tensor (the experts' weights
+  // stacked along rows)
+  const int* tile_group;
+  int group_rows;
   int k_splits;  // 1 = off
   int total_kb;  // host side: the smallest K-block total of any tile (bounds the split count)
   float4* split_ws;  // [tiles * k_splits][BN / 4][128]
@@ -496,6 +503,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int tile = cluster; tile < num_tiles; tile += clusters) {
         int tm, tn;
         tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+        int grp_off = 0;
+        if (g.tile_group) {
+          const int grp = g.tile_group[tm];
+          if (grp < 0) continue;
+          grp_off = grp * g.group_rows;
+        }
         const int m0 = tm * 2 * kBM + static_cast<int>(rank) * kBM;
         const int n0 = tn * BN + static_cast<int>(rank) * kHalfN;
         const int reg0 = region_of(g, tn * BN);
@@ -512,11 +525,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const int n = n0 + (i < nbox ? i : 0) * box_n;
             if (g.b_by_rank) {
               bmap[i] = &g.maps[sg.b_map[rank]];
-              bcoord[i] = tn * kHalfN + (i < nbox ? i : 0) * box_n;
+              bcoord[i] = tn * kHalfN + (i < nbox ? i : 0) * box_n + grp_off;
             } else {
               const int r = region_of(g, n);
               bmap[i] = &g.maps[sg.b_map[r]];
-              bcoord[i] = n - g.region_n0[r];
+              bcoord[i] = n - g.region_n0[r] + grp_off;
             }
           }
           const uint32_t box_bytes = static_cast<uint32_t>(box_n) * kBK * 2;
@@ -556,6 +569,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = cluster; tile < num_tiles; tile += clusters) {
+        if (g.tile_group) {
+          int tm, tn;
+          tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+          if (g.tile_group[tm] < 0) continue;
+        }
         mbar_wait(&tempty[acc], acc_phase ^ 1u, wg);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -596,6 +614,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = cluster; tile < num_tiles; tile += clusters) {
       int tm, tn;
       tile_coords(tile, g.tiles_m, g.tiles_n, tm, tn);
+      if (g.tile_group && g.tile_group[tm] < 0) continue;
       mbar_wait(&tfull[acc], acc_phase, wg);
       tc_fence_after();
       const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * BN) + (static_cast<uint32_t>(quarter * 32) << 16);

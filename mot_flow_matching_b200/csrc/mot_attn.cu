@@ -1774,3 +1774,6 @@ mot_status mot_dev_saved_layout(const mot_attn_config* cfg, int32_t batch, int32
 
 // ------------------------------------------------------------------ the denoise step
 #include "mot_step.cuh"
+
+// ------------------------------------------------------------------ the A3B mixture-of-experts MLP
+#include "mot_moe.cuh"
