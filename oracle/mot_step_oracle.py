@@ -36,6 +36,12 @@ Readings where the pages give no formula:
      (t_eps keeps the division away from sigma = 0).
   S6 shifted schedule: sigma_i = shift u_i / (1 + (shift - 1) u_i),
      u_i = 1 - i / steps, i = 0..steps.
+  S7 bf16 exchange points: the tower is a bf16 model (bf16 weights, bf16
+     GEMM operands), so every GEMM input that the step forms itself is one
+     round-to-nearest-even bf16 value: the patch tokens entering the
+     embedding, RMSNorm(h) g entering each attention and MLP half, and the
+     normed state entering the head. The residual stream h and the Euler
+     update stay in full precision (z there is the unrounded input).
 """
 from __future__ import annotations
 
@@ -43,7 +49,7 @@ from typing import Dict, Sequence
 
 import numpy as np
 
-from oracle.mot_attn_oracle import layer_forward
+from oracle.mot_attn_oracle import layer_forward, round_to_bf16
 from oracle.mot_mlp_oracle import mlp_forward
 
 
@@ -92,17 +98,17 @@ def denoise_step(z: np.ndarray, model: Dict, layers: Sequence[Dict], caches: Seq
     v_cache [B, Hkv, P, dh]. Returns z_next [N, C] and the per-branch x0.
     """
     nb = len(prefix_len)
-    h0 = z @ model["w_in"].T + timestep_embedding(sigma, model["w_in"].shape[0])
+    h0 = round_to_bf16(z) @ model["w_in"].T + timestep_embedding(sigma, model["w_in"].shape[0])  # S2, S7
     h = np.repeat(h0[None], nb, axis=0)
     for lw, cache in zip(layers, caches):
         attn_in = dict(lw)
-        attn_in["x"] = rms_norm_rows(h, lw["norm_in"], eps)
+        attn_in["x"] = round_to_bf16(rms_norm_rows(h, lw["norm_in"], eps))  # S1, S7
         attn_in["k_cache"], attn_in["v_cache"] = cache["k_cache"], cache["v_cache"]
         attn_in["prefix_len"] = np.asarray(prefix_len)
         h = h + layer_forward(attn_in, attn_dims, lora_scale)["y"]
         mw = {k[4:]: v for k, v in lw.items() if k.startswith("mlp_")}
-        h = h + np.stack([mlp_forward(rms_norm_rows(h[b], lw["norm_post"], eps), mw, lora_scale)["y"]
-                          for b in range(nb)])
-    x0 = rms_norm_rows(h, model["norm_out"], eps) @ model["w_out"].T
+        h = h + np.stack([mlp_forward(round_to_bf16(rms_norm_rows(h[b], lw["norm_post"], eps)), mw,
+                                      lora_scale)["y"] for b in range(nb)])
+    x0 = round_to_bf16(rms_norm_rows(h, model["norm_out"], eps)) @ model["w_out"].T  # S3, S7
     xg = guidance(x0, cfg, img_cfg)
     return {"z_next": euler_update(z, xg, sigma, sigma_next, t_eps), "x0": x0, "h": h}

@@ -92,8 +92,8 @@ def test_step_residual_identity():
         w["w_o"] = np.zeros_like(w["w_o"])
         w["mlp_w_down"] = np.zeros_like(w["mlp_w_down"])
     res = SO.denoise_step(z, model, lw, caches, [3, 2], O.dims_of(wl), 0.0, 0.6, 0.4, 4.0, 1.0, 0.02)
-    h0 = z @ model["w_in"].T + SO.timestep_embedding(0.6, wl.dims.hidden)
-    x0 = SO.rms_norm_rows(h0, model["norm_out"], 1e-6) @ model["w_out"].T
+    h0 = O.round_to_bf16(z) @ model["w_in"].T + SO.timestep_embedding(0.6, wl.dims.hidden)
+    x0 = O.round_to_bf16(SO.rms_norm_rows(h0, model["norm_out"], 1e-6)) @ model["w_out"].T
     np.testing.assert_allclose(res["h"][0], h0, rtol=0, atol=1e-12)
     np.testing.assert_allclose(res["z_next"], z + (0.4 - 0.6) * (z - x0) / 0.6, rtol=0, atol=1e-12)
 
@@ -125,3 +125,35 @@ def test_step_norm_gains_feed_their_own_half():
     np.testing.assert_allclose(a["h"], b["h"], rtol=0, atol=1e-12)
     full = SO.denoise_step(z, model, lw, caches, *args)
     assert not np.allclose(full["h"], a["h"])
+
+
+def test_step_gemm_inputs_are_bf16_and_euler_uses_the_exact_z(monkeypatch):
+    # S7: every input the step hands to a layer is a bf16 value (within half a
+    # bf16 ulp of the unrounded norm), while the Euler update keeps the exact
+    # z: moving z inside its bf16 rounding cell leaves x0 unchanged and moves
+    # z_next by (z - z') sigma_next / sigma
+    seen = []
+    real_attn, real_mlp = SO.layer_forward, SO.mlp_forward
+
+    def attn_spy(inp, dims, s):
+        seen.append(inp["x"])
+        return real_attn(inp, dims, s)
+
+    def mlp_spy(x, w, s):
+        seen.append(x)
+        return real_mlp(x, w, s)
+
+    monkeypatch.setattr(SO, "layer_forward", attn_spy)
+    monkeypatch.setattr(SO, "mlp_forward", mlp_spy)
+    wl, model, lw, caches, z = _tiny_model(7, rank=2)
+    args = ([3, 2], O.dims_of(wl), 1.0, 0.8, 0.6, 4.0, 1.0, 0.02)
+    a = SO.denoise_step(z, model, lw, caches, *args)
+    assert len(seen) == len(lw) * (1 + len(args[0]))  # one attention call, one MLP call per branch
+    for x in seen:
+        assert np.array_equal(O.round_to_bf16(x), x)
+    assert all(np.any(x != 0) for x in seen)
+    z2 = O.round_to_bf16(z)
+    assert not np.array_equal(z2, z)
+    b = SO.denoise_step(z2, model, lw, caches, *args)
+    np.testing.assert_array_equal(a["x0"], b["x0"])
+    np.testing.assert_allclose(a["z_next"] - b["z_next"], (z - z2) * 0.6 / 0.8, rtol=0, atol=1e-14)
