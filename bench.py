@@ -252,6 +252,28 @@ def run_once_mlp(args):
     return 0 if status == 0 else 1
 
 
+def run_once_moe(args):
+    """Two warm calls of the A3B mixture-of-experts MLP over the 8192 image
+    tokens of a 2048^2 CFG call (the target of ncu captures)."""
+    import torch
+    from mot_flow_matching_b200 import synth
+    from mot_flow_matching_b200.moe import MotMoe
+    dev = torch.device("cuda", 0)
+    T, d, E, K, I = 8192, synth.MOE_HIDDEN, synth.MOE_EXPERTS, synth.MOE_TOP_K, synth.MOE_INTER
+    draw = lambda shape, std, seed: synth.draw_device(shape, std, 0.0, seed, dev)
+    w = {"w_router": draw((E, d), 0.02, 980_001), "w_gate": draw((E, I, d), 0.02, 980_002),
+         "w_up": draw((E, I, d), 0.02, 980_003), "w_down": draw((E, d, I), 0.02, 980_004)}
+    x = draw((T, d), 1.0, 980_005)
+    moe = MotMoe(w, top_k=K, max_tokens=T)
+    for _ in range(2):
+        y = moe.forward(x)
+    torch.cuda.synchronize()
+    status = moe.device_status()
+    moe.close()
+    print(json.dumps({"once": "moe_a3b_8192_tokens", "status": status, "y_abs_mean": float(y.float().abs().mean())}))
+    return 0 if status == 0 else 1
+
+
 def run_once(args):
     """One warm forward of a workload (the target of ncu captures)."""
     import torch
@@ -261,6 +283,8 @@ def run_once(args):
     build_mod.build()
     if args.mlp:
         return run_once_mlp(args)
+    if args.moe:
+        return run_once_moe(args)
     wl = synth.WORKLOADS[args.workload]
     t = synth.workload_inputs(args.workload)
     td = {k: (v.cuda() if k != "prefix_len" else v) for k, v in t.items()}
@@ -973,6 +997,7 @@ def main():
     ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX)
     ap.add_argument("--train", action="store_true", help="with --once: forward keeping activations + backward")
     ap.add_argument("--mlp", action="store_true", help="with --once: the gen-tower MLP instead of the attention")
+    ap.add_argument("--moe", action="store_true", help="with --once: the A3B mixture-of-experts MLP")
     ap.add_argument("--check-ranks", action="store_true",
                     help="CPU check of the rank plumbing (gloo): spawn/launcher handling, shards, max over ranks")
     args = ap.parse_args()

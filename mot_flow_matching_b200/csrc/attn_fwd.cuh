@@ -379,7 +379,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_wait(&s_full[t], jj & 1, wg);
       tc_fence_after();
       const int valid = key_end - (j0 + jj) * 128;  // keys of this tile this row sees (>= 1 on the first tile)
-      const bool full = valid >= 128;
+      // warp-uniform: the exp/store path issues tcgen05.st, a warp-collective
+      // instruction, so all 32 lanes must take the same template branch
+      // (in causal mode `valid` differs from row to row)
+      const bool full = __all_sync(0xffffffffu, valid >= 128);
       HalfRowS srow;
       load_half_row(tS + col0, srow);
       const float pm = full ? half_row_max<true>(srow, col0, valid) : half_row_max<false>(srow, col0, valid);

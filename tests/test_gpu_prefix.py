@@ -34,15 +34,26 @@ def _run(wl, t, lengths):
 
 def _check_cache(got_bf16, ref64, lengths, what):
     # one rounding to bf16 of an f32 value that is within f32 error of the
-    # fp64 one: at most one bf16 ulp from the oracle's rounded value
+    # fp64 one: at most one bf16 ulp from the oracle's rounded value plus that
+    # f32 error, and equal to it almost everywhere. The f32 error is absolute
+    # (a K = 4096 dot product accumulates about sqrt(K) 2^-24 sum|x w|, some
+    # 1e-4 of the RMS), so near-zero entries, whose ulp is tiny, get the floor
+    # tau = 2^-10 RMS. (A max bar relative to the RMS does not fit a bf16
+    # result: half an ulp of an element at 4x the RMS is already 1.6e-2 of the
+    # RMS.) The mean bar still applies.
     for b, n in enumerate(lengths):
         g = got_bf16[b][:, :n].double().cpu().numpy()
         r = ref64[b][:, :n]
-        assert_parity(g, r, f"{what} branch {b}", max_tol=1.2e-2, mean_tol=2e-3)
+        assert_parity(g, r, f"{what} branch {b}", max_tol=np.inf, mean_tol=2e-3)
         rb = PO.cache_bf16(r)
         _, e = np.frexp(r)
         ulp = np.ldexp(1.0, e - 8)
-        assert np.all(np.abs(g - rb) <= ulp * 1.0001), what
+        tau = 2.0 ** -10 * np.sqrt(np.mean(r * r))
+        bad = np.abs(g - rb) > ulp * 1.0001 + tau
+        if bad.any():
+            i = np.unravel_index(np.argmax(np.abs(g - rb) - ulp), g.shape)
+            raise AssertionError(f"{what} branch {b}: {int(bad.sum())} entries off by more than one ulp + tau; "
+                                 f"worst at {i}: got {g[i]!r} oracle {r[i]!r} rounded {rb[i]!r} tau {tau:.3e}")
         assert np.mean(g != rb) < 0.01, (what, np.mean(g != rb))
 
 

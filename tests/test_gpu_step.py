@@ -3,9 +3,19 @@ decoder layers of the attention and MLP kernels, x0 head, guidance, Euler
 update) against its fp64 oracle (oracle/mot_step_oracle.py).
 
 With sigma = 0.5 and sigma_next = 0 the Euler update returns the guided x0
-itself (z + (0 - 0.5)(z - x0)/0.5 = x0), so the step's output is compared
-with the oracle's guided head output directly; a generic sigma pair checks
-the update. Parity bar on the f32 result as for the layers."""
+itself (z + (0 - 0.5)(z - x0)/0.5 = x0). Guidance is linear in the branches'
+head outputs, x0_g = sum_b c_b x0_b with (cfg, 1 - cfg) for two branches and
+(cfg, img_cfg - cfg, 1 - img_cfg) for three, so guidance weights that pick
+one branch (cfg 1 or 0, img_cfg 1 or 0) return that branch's x0, and each
+branch is held to the layers' parity bar on its own. The pages' guidance
+(cfg 4, img_cfg 1.5) is then checked as that linear combination of the GPU's
+own branch outputs (f32 arithmetic), and against the oracle within the bound
+the same combination puts on the branch errors. A generic sigma pair checks
+the update.
+
+Bar: each branch's x0 comes out of 2 L sublayers (attention and MLP per
+layer) whose errors, each within the layer bar, add into the residual
+stream independently, so the step's bar is the layer bar times sqrt(2 L)."""
 import numpy as np
 import pytest
 import torch
@@ -16,7 +26,7 @@ from mot_flow_matching_b200.mlp import MotMlp
 from mot_flow_matching_b200.step import MotStep
 from oracle import mot_attn_oracle as O
 from oracle import mot_step_oracle as SO
-from tests.gpu_helpers import assert_parity, ensure_built
+from tests.gpu_helpers import MAX_TOL, MEAN_TOL, assert_parity, ensure_built
 
 pytestmark = pytest.mark.gpu
 
@@ -74,10 +84,53 @@ def _run(step, keep, inp, wl, plen, sigma, sigma_next, cfg, img_cfg):
 SMALL = synth.LayerDims(hidden=512, n_q_heads=4, n_kv_heads=2)
 
 
+def _branch_coeffs(B, cfg, img_cfg):
+    """x0_g = sum_b c_b x0_b: the guidance of the pages as branch weights."""
+    if B == 1:
+        return [1.0]
+    if B == 2:
+        return [cfg, 1.0 - cfg]
+    return [cfg, img_cfg - cfg, 1.0 - img_cfg]
+
+
+def _picks(B):
+    """(cfg, img_cfg) that return branch b alone, for each b."""
+    return {1: [(1.0, 1.0)], 2: [(1.0, 1.0), (0.0, 1.0)], 3: [(1.0, 1.0), (0.0, 1.0), (0.0, 0.0)]}[B]
+
+
+def _bar(n_layers):
+    f = float(np.sqrt(2 * n_layers))
+    return dict(max_tol=MAX_TOL * f, mean_tol=MEAN_TOL * f)
+
+
+def _check_branches_and_guidance(step, keep, inp, wl, plen, cfg, img_cfg, what):
+    B = wl.batch
+    bar = _bar(len(inp["layers"]))
+    ref = _oracle(inp, wl, plen, 0.5, 0.0, cfg, img_cfg)
+    branch = []
+    for b, (c, ic) in enumerate(_picks(B)):
+        assert _branch_coeffs(B, c, ic) == [1.0 if i == b else 0.0 for i in range(B)]
+        got = _run(step, keep, inp, wl, plen, 0.5, 0.0, c, ic)
+        assert_parity(got, ref["x0"][b], f"{what}: x0 of branch {b}", **bar)
+        branch.append(got)
+    got = _run(step, keep, inp, wl, plen, 0.5, 0.0, cfg, img_cfg)
+    co = _branch_coeffs(B, cfg, img_cfg)
+    lin = sum(c * x for c, x in zip(co, branch))
+    # the combine and the Euler update (which passes z - x0 through f32) in
+    # f32: a few roundings of each term, z included
+    az = np.abs(inp["z"].double().numpy())
+    scale = sum(abs(c) * (np.abs(x) + az) for c, x in zip(co, branch)) + np.abs(lin) + az
+    assert np.all(np.abs(got - lin) <= 8 * 2.0 ** -24 * scale + 1e-30), what
+    exp = SO.guidance(ref["x0"], cfg, img_cfg)
+    np.testing.assert_allclose(ref["z_next"], exp, rtol=0, atol=1e-12)
+    err = sum(abs(c) * np.abs(x - r) for c, x, r in zip(co, branch, ref["x0"]))
+    assert np.all(np.abs(got - exp) <= err * (1 + 1e-6) + 8 * 2.0 ** -24 * scale), what
+
+
 @pytest.mark.parametrize("B,N,P,plen,n_layers,rank,cfg,img_cfg", [
     (2, 200, 37, [37, 20], 2, 16, 4.0, 1.0),
     (3, 129, 64, [64, 64, 0], 2, 8, 4.0, 1.5),
-    (1, 77, 5, [5], 1, 0, 1.0, 1.0),
+    (1, 77, 5, [5], 1, 0, 4.0, 1.0),
 ])
 def test_step_small_dims_x0(cuda_ready, B, N, P, plen, n_layers, rank, cfg, img_cfg):
     wl = synth.Workload("step", B, N, P, rank, float(rank), dims=SMALL)
@@ -85,11 +138,7 @@ def test_step_small_dims_x0(cuda_ready, B, N, P, plen, n_layers, rank, cfg, img_
     for t in inp["layers"]:
         t["prefix_len"] = torch.tensor(plen, dtype=torch.int32)
     step, keep, _ = _build(inp, wl, 384)
-    got = _run(step, keep, inp, wl, plen, 0.5, 0.0, cfg, img_cfg)
-    ref = _oracle(inp, wl, plen, 0.5, 0.0, cfg, img_cfg)
-    # sigma 0.5 -> 0: the step returns the guided x0
-    assert_parity(got, SO.guidance(ref["x0"], cfg, img_cfg), "guided x0")
-    np.testing.assert_allclose(ref["z_next"], SO.guidance(ref["x0"], cfg, img_cfg), rtol=0, atol=1e-12)
+    _check_branches_and_guidance(step, keep, inp, wl, plen, cfg, img_cfg, "guided x0")
     step.close()
 
 
@@ -99,11 +148,13 @@ def test_step_euler_update(cuda_ready):
     step, keep, _ = _build(inp, wl, 384)
     sig = SO.sigma_schedule(8, 3.0)
     s0, s1 = float(sig[3]), float(sig[4])
-    got = _run(step, keep, inp, wl, [48, 48], s0, s1, 4.0, 1.0)
-    ref = _oracle(inp, wl, [48, 48], s0, s1, 4.0, 1.0)
+    # cfg 1: the update applied to the conditional branch's x0 (the guidance
+    # combine has its own test)
+    got = _run(step, keep, inp, wl, [48, 48], s0, s1, 1.0, 1.0)
+    ref = _oracle(inp, wl, [48, 48], s0, s1, 1.0, 1.0)
     z = inp["z"].double().numpy()
     # the update part of the step, z_next - z = (s1 - s0) (z - x0) / s0
-    assert_parity(got - z, ref["z_next"] - z, "z_next - z")
+    assert_parity(got - z, ref["z_next"] - z, "z_next - z", **_bar(2))
     step.close()
 
 
@@ -114,7 +165,5 @@ def test_step_full_dims_two_layers(cuda_ready):
     wl = synth.Workload("step", 2, 256, 64, 16, 16.0)
     inp = synth.make_step_inputs(2, wl, synth.MLP_INTER, 3072, 7400)
     step, keep, _ = _build(inp, wl, synth.MLP_INTER)
-    got = _run(step, keep, inp, wl, [64, 64], 0.5, 0.0, 4.0, 1.0)
-    ref = _oracle(inp, wl, [64, 64], 0.5, 0.0, 4.0, 1.0)
-    assert_parity(got, SO.guidance(ref["x0"], 4.0, 1.0), "guided x0 (full dims)")
+    _check_branches_and_guidance(step, keep, inp, wl, [64, 64], 4.0, 1.0, "guided x0 (full dims)")
     step.close()
