@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the 2048^2 CFG workload, keyed by the sha256 of the
 # kernel's source file at capture time: a changed kernel reports null.
 TRAFFIC = {
-    "attn_fwd": {"sha256": "bdc599b623238d957f063bc5acac4a7266ff1705f724d6ff19c0fb05ebd75e5d",
-                 "bytes": 104960512 + 33044224},
+    "attn_fwd": {"sha256": "f35c17d939924ee887ac497ea302c33107340a8f3b9650d1cb8c6f22c4442d80",
+                 "bytes": 105389568 + 32933376},
     "qkv_gemm": {"sha256": "9cc99ea8dda5aee19ed56221282f43d36bd6c96740405226bbd7867286c344cf",
                  "bytes": 221264128 + 81383936},
 }
