@@ -60,7 +60,10 @@ mot_status mot_moe_create(const mot_moe_config* cfg, const mot_moe_weights* weig
  *           token in rank order (for checks of the routing)
  *   workspace device, workspace_bytes from mot_moe_query_workspace
  * The expert GEMMs run on M tiles of 256 rows of one expert each; their
- * count depends on the routing and is bounded by ceil(T top_k / 256) + E. */
+ * count depends on the routing and is bounded by ceil(T top_k / 256) + E.
+ * The experts' activations h and outputs are kept in f16 between the
+ * kernels; an overflow there is latched as MOT_ERR_NUMERIC and reported by
+ * mot_moe_get_device_status. */
 mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t tokens, void* y, float* y_f32, int32_t* experts_out,
                            void* workspace, size_t workspace_bytes, void* stream);
 

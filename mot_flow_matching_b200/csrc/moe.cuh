@@ -20,58 +20,49 @@ constexpr int kMoeTileRows = 256;
 
 // Softmax over the E router logits of each token, its top_k experts (ties to
 // the lower index) and their probabilities renormalised to sum to one; one
-// warp per token, lane e holds expert e. counts[e] gains one per selection.
+// warp per token, lane e holds expert e. Each lane finds its expert's rank
+// directly (how many experts have a larger logit, or an equal one at a lower
+// index: the order of the probabilities, which exp keeps), so the selection
+// has no dependent rounds; the lanes ranked below top_k write their slot.
+// counts[e] gains one per selection (summed per block in shared memory).
 __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict__ logits, int T, int E, int K,
                                                         int* __restrict__ topk_idx, float* __restrict__ topk_w,
                                                         int* __restrict__ counts) {
+  __shared__ int block_counts[kMoeMaxExperts];
+  if (threadIdx.x < kMoeMaxExperts) block_counts[threadIdx.x] = 0;
+  __syncthreads();
   grid_dep_launch();
   grid_dep_wait();
   const int lane = threadIdx.x & 31;
+  const bool live = lane < E;
   const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
   for (int t = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < T; t += nwarps) {
-    const float v = lane < E ? logits[static_cast<long long>(t) * E + lane] : -INFINITY;
+    const float v = live ? logits[static_cast<long long>(t) * E + lane] : -INFINITY;
     float m = v;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float p = lane < E ? expf(v - m) : 0.f;
+    float p = live ? expf(v - m) : 0.f;
     float s = p;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    p = lane < E ? p / s : -1.f;  // unselectable below any probability
-    int sel[kMoeMaxTopK];
-    float w[kMoeMaxTopK];
-    float wsum = 0.f;
-#pragma unroll
-    for (int k = 0; k < kMoeMaxTopK; ++k) {
-      if (k >= K) break;
-      // largest p, then the lowest lane: probabilities are >= 0, so their
-      // bit patterns order as unsigned integers
-      unsigned hi = p >= 0.f ? __float_as_uint(p) : 0u;
-      unsigned lo = static_cast<unsigned>(31 - lane);
-      if (p < 0.f) lo = 0u;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned ohi = __shfl_xor_sync(0xffffffffu, hi, o);
-        const unsigned olo = __shfl_xor_sync(0xffffffffu, lo, o);
-        if (ohi > hi || (ohi == hi && olo > lo)) {
-          hi = ohi;
-          lo = olo;
-        }
-      }
-      sel[k] = 31 - static_cast<int>(lo);
-      w[k] = __uint_as_float(hi);
-      wsum += w[k];
-      if (lane == sel[k]) p = -1.f;
+    p = p / s;
+    int rank = 0;
+    for (int j = 0; j < E; ++j) {
+      const float vj = __shfl_sync(0xffffffffu, v, j);
+      rank += (vj > v || (vj == v && j < lane)) ? 1 : 0;
     }
-    if (lane == 0) {
-      const float inv = 1.0f / wsum;
-      for (int k = 0; k < K; ++k) {
-        topk_idx[static_cast<long long>(t) * K + k] = sel[k];
-        topk_w[static_cast<long long>(t) * K + k] = w[k] * inv;
-        atomicAdd(&counts[sel[k]], 1);
-      }
+    const bool sel = live && rank < K;
+    float ws = sel ? p : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+    if (sel) {
+      topk_idx[static_cast<long long>(t) * K + rank] = lane;
+      topk_w[static_cast<long long>(t) * K + rank] = p / ws;
+      atomicAdd(&block_counts[lane], 1);
     }
   }
+  __syncthreads();
+  if (threadIdx.x < E && block_counts[threadIdx.x] > 0) atomicAdd(&counts[threadIdx.x], block_counts[threadIdx.x]);
 }
 
 // Expert block offsets (each count padded to a multiple of 256), the M-tile
@@ -105,11 +96,12 @@ __global__ void moe_offsets_kernel(const int* __restrict__ counts, int E, int ti
   }
 }
 
-// Gathers each token's row into the slot of every expert it was routed to
+// Copies each token's row into the slot of every expert it was routed to
 // (slot order within an expert follows arrival; every row of an expert's
 // GEMM is computed independently, so the block's result does not depend on
 // it) and records the slot per (token, rank); then zeroes the padding rows
-// of every expert block. One warp per row.
+// of every expert block. One warp per token: lanes 0..K-1 claim the K slots
+// at once, and the row is read once and written K times.
 __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* __restrict__ x, int T, int K, int d,
                                                            const int* __restrict__ topk_idx,
                                                            const int* __restrict__ offsets,
@@ -123,18 +115,27 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* 
   const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
   const int warp0 = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int n16 = d / 8;  // 16-byte chunks per row
-  for (int pr = warp0; pr < T * K; pr += nwarps) {
-    const int t = pr / K;
+  for (int t = warp0; t < T; t += nwarps) {
     int pos = 0;
-    if (lane == 0) {
+    if (lane < K) {
+      const long long pr = static_cast<long long>(t) * K + lane;
       const int e = topk_idx[pr];
       pos = offsets[e] + atomicAdd(&fill[e], 1);
       slot[pr] = pos;
     }
-    pos = __shfl_sync(0xffffffffu, pos, 0);
+    uint4* dst[kMoeMaxTopK];
+#pragma unroll
+    for (int k = 0; k < kMoeMaxTopK; ++k)
+      dst[k] = reinterpret_cast<uint4*>(xp + static_cast<long long>(__shfl_sync(0xffffffffu, pos, k)) * d);
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(t) * d);
-    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<long long>(pos) * d);
-    for (int c = lane; c < n16; c += 32) dst[c] = src[c];
+    for (int c = lane; c < n16; c += 32) {
+      const uint4 v = src[c];
+#pragma unroll
+      for (int k = 0; k < kMoeMaxTopK; ++k) {
+        if (k >= K) break;
+        dst[k][c] = v;
+      }
+    }
   }
   const int rows = *total_rows;
   for (int r = warp0; r < rows; r += nwarps) {
@@ -145,9 +146,10 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* 
   }
 }
 
-// y[t] = sum over ranks k (in order) of w[t, k] * yp[slot[t, k]]: f32 and
-// bf16 = RNE(f32). One warp per token, d a multiple of 128.
-__global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ yp, int T, int K, int d,
+// y[t] = sum over ranks k (in order) of w[t, k] * yp[slot[t, k]] (yp: the f16
+// expert outputs): f32 and bf16 = RNE(f32). One warp per token, d a multiple
+// of 128.
+__global__ void __launch_bounds__(256) moe_combine_kernel(const __half* __restrict__ yp, int T, int K, int d,
                                                           const int* __restrict__ slot,
                                                           const float* __restrict__ topk_w,
                                                           __nv_bfloat16* __restrict__ y, float* __restrict__ y32) {
@@ -156,16 +158,26 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
   const int lane = threadIdx.x & 31;
   const int nwarps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
   for (int t = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < T; t += nwarps) {
+    int sl[kMoeMaxTopK];
+    float wk[kMoeMaxTopK];
+#pragma unroll
+    for (int k = 0; k < kMoeMaxTopK; ++k) {
+      const long long pr = static_cast<long long>(t) * K + k;
+      sl[k] = k < K ? slot[pr] : 0;
+      wk[k] = k < K ? topk_w[pr] : 0.f;
+    }
     for (int c = lane * 4; c < d; c += 128) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int k = 0; k < K; ++k) {
-        const long long pr = static_cast<long long>(t) * K + k;
-        const float wk = topk_w[pr];
-        const float4 v = *reinterpret_cast<const float4*>(yp + static_cast<long long>(slot[pr]) * d + c);
-        acc.x = fmaf(wk, v.x, acc.x);
-        acc.y = fmaf(wk, v.y, acc.y);
-        acc.z = fmaf(wk, v.z, acc.z);
-        acc.w = fmaf(wk, v.w, acc.w);
+#pragma unroll
+      for (int k = 0; k < kMoeMaxTopK; ++k) {
+        if (k >= K) break;
+        const uint2 raw = *reinterpret_cast<const uint2*>(yp + static_cast<long long>(sl[k]) * d + c);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        acc.x = fmaf(wk[k], a.x, acc.x);
+        acc.y = fmaf(wk[k], a.y, acc.y);
+        acc.z = fmaf(wk[k], b.x, acc.z);
+        acc.w = fmaf(wk[k], b.y, acc.w);
       }
       const long long o = static_cast<long long>(t) * d + c;
       if (y32) *reinterpret_cast<float4*>(y32 + o) = acc;

@@ -9,8 +9,8 @@
 //   moe_dispatch     x rows gathered into their experts' slots, padding zeroed
 //   gate/up GEMM     grouped CTA pairs (rank 0 W_gate rows, rank 1 W_up rows
 //                    of the tile's expert) with the SwiGLU epilogue -> f16 h
-//   down GEMM        grouped CTA pairs, h W_down^T (f16 copy) -> f32 per slot
-//   moe_combine      y = sum_k w_k (slot rows), f32 and bf16
+//   down GEMM        grouped CTA pairs, h W_down^T (f16 copy) -> f16 per slot
+//   moe_combine      y = sum_k w_k (slot rows) in f32; f32 and bf16 out
 #pragma once
 
 #include "mot_moe.h"
@@ -54,7 +54,7 @@ MoeLayout make_moe_layout(const mot_moe_config& c, int T) {
   L.slot = take(t * K * 4);
   L.xp = take(static_cast<size_t>(L.rows) * d * 2);
   L.hp = take(static_cast<size_t>(L.rows) * I * 2);
-  L.yp = take(static_cast<size_t>(L.rows) * d * 4);
+  L.yp = take(static_cast<size_t>(L.rows) * d * 2);
   L.total = off;
   return L;
 }
@@ -178,7 +178,7 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   int* slot = reinterpret_cast<int*>(ws + L.slot);
   __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(ws + L.xp);
   __half* hp = reinterpret_cast<__half*>(ws + L.hp);
-  float* yp = reinterpret_cast<float*>(ws + L.yp);
+  __half* yp = reinterpret_cast<__half*>(ws + L.yp);
   const int d = c.hidden, I = c.intermediate, E = c.experts, K = c.top_k;
   cudaError_t e = cudaMemsetAsync(counts, 0, kMoeMaxExperts * sizeof(int), st);
   // router logits
@@ -202,7 +202,7 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   if (e == cudaSuccess)
     e = launch_pdl(moe_offsets_kernel, dim3(1), dim3(256), 0, st, static_cast<const int*>(counts), E, L.tiles, offsets,
                    tile_expert, total_rows, fill);
-  const int disp_grid = std::max(1, std::min((T * K + 7) / 8, 16 * h->num_sms));
+  const int disp_grid = std::max(1, std::min((T + 7) / 8, 16 * h->num_sms));
   if (e == cudaSuccess)
     e = launch_pdl(moe_dispatch_kernel, dim3(disp_grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), T, K,
                    d, static_cast<const int*>(idx), static_cast<const int*>(offsets), static_cast<const int*>(counts),
@@ -224,7 +224,7 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
     EpiSwiGLU::Params ep{hp, nullptr, nullptr, L.rows, I};
     e = launch_gemm2<256, 6, EpiSwiGLU>(core, ep, h->num_sms, st);
   }
-  // down projection of every slot's expert -> f32 slot rows
+  // down projection of every slot's expert -> f16 slot rows (overflow latched)
   if (e == cudaSuccess) {
     GemmCore core;
     core_init(core, L.rows, d, 256, 128, h->status);
@@ -236,12 +236,12 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
     core.segs[0] = seg1(0, 0, 2, I / 64, idesc_f16(256, 256, false, false), false, false);
     core.num_segs = 1;
     EpiStore::Params ep = store_params(L.rows, d);
-    ep.out32 = yp;
-    ep.ld32 = d;
+    set_out16(ep, 0, yp, d, false);
+    ep.check_f16 = 1;
     e = launch_gemm2<256, 6, EpiStore>(core, ep, h->num_sms, st);
   }
   if (e == cudaSuccess)
-    e = launch_pdl(moe_combine_kernel, dim3(warps_grid), dim3(256), 0, st, static_cast<const float*>(yp), T, K, d,
+    e = launch_pdl(moe_combine_kernel, dim3(warps_grid), dim3(256), 0, st, static_cast<const __half*>(yp), T, K, d,
                    static_cast<const int*>(slot), static_cast<const float*>(wts), static_cast<__nv_bfloat16*>(y),
                    y_f32);
   if (e == cudaSuccess && experts_out)
