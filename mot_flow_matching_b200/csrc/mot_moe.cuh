@@ -2,10 +2,10 @@
 // include/mot_moe.h). Same translation unit as mot_attn.cu.
 //
 // Launch sequence on the caller's stream (T tokens, E experts, top K, width I):
-//   memset           expert counts
 //   router GEMM      logits = x W_r^T (f32 [T, E]), 1-CTA, split-K
-//   moe_route        softmax, top K, renormalised weights, counts
-//   moe_offsets      expert blocks padded to 256 rows, M-tile -> expert table
+//   moe_route        softmax, top K, renormalised weights, per-block numbering
+//   moe_offsets      per-expert scan over the routing blocks, expert blocks
+//                    padded to 256 rows, M-tile -> expert table
 //   moe_dispatch     x rows gathered into their experts' slots, padding zeroed
 //   gate/up GEMM     grouped CTA pairs (rank 0 W_gate rows, rank 1 W_up rows
 //                    of the tile's expert) with the SwiGLU epilogue -> f16 h
@@ -31,8 +31,9 @@ struct mot_moe {
 namespace {
 
 struct MoeLayout {
-  int tiles = 0, rows = 0;
-  size_t logits = 0, idx = 0, wts = 0, small = 0, tile_expert = 0, slot = 0, xp = 0, hp = 0, yp = 0, total = 0;
+  int tiles = 0, rows = 0, nblk = 0;
+  size_t logits = 0, idx = 0, wts = 0, pos = 0, blk_cnt = 0, blk_base = 0, small = 0, tile_expert = 0, slot = 0,
+         xp = 0, hp = 0, yp = 0, total = 0;
 };
 
 MoeLayout make_moe_layout(const mot_moe_config& c, int T) {
@@ -40,6 +41,7 @@ MoeLayout make_moe_layout(const mot_moe_config& c, int T) {
   const size_t d = c.hidden, I = c.intermediate, E = c.experts, K = c.top_k, t = T;
   L.tiles = static_cast<int>((t * K + kMoeTileRows - 1) / kMoeTileRows + E);
   L.rows = L.tiles * kMoeTileRows;
+  L.nblk = static_cast<int>((t + kMoeRouteTokens - 1) / kMoeRouteTokens);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -49,7 +51,10 @@ MoeLayout make_moe_layout(const mot_moe_config& c, int T) {
   L.logits = take(t * E * 4);
   L.idx = take(t * K * 4);
   L.wts = take(t * K * 4);
-  L.small = take(4 * kMoeMaxExperts * 4);  // counts, fill, offsets, total rows
+  L.pos = take(t * K * 4);
+  L.blk_cnt = take(static_cast<size_t>(L.nblk) * E * 4);
+  L.blk_base = take(static_cast<size_t>(L.nblk) * E * 4);
+  L.small = take(3 * kMoeMaxExperts * 4);  // counts, offsets, total rows
   L.tile_expert = take(static_cast<size_t>(L.tiles) * 4);
   L.slot = take(t * K * 4);
   L.xp = take(static_cast<size_t>(L.rows) * d * 2);
@@ -170,9 +175,11 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   float* logits = reinterpret_cast<float*>(ws + L.logits);
   int* idx = reinterpret_cast<int*>(ws + L.idx);
   float* wts = reinterpret_cast<float*>(ws + L.wts);
+  int* pos = reinterpret_cast<int*>(ws + L.pos);
+  int* blk_cnt = reinterpret_cast<int*>(ws + L.blk_cnt);
+  int* blk_base = reinterpret_cast<int*>(ws + L.blk_base);
   int* counts = reinterpret_cast<int*>(ws + L.small);
-  int* fill = counts + kMoeMaxExperts;
-  int* offsets = fill + kMoeMaxExperts;
+  int* offsets = counts + kMoeMaxExperts;
   int* total_rows = offsets + kMoeMaxExperts;
   int* tile_expert = reinterpret_cast<int*>(ws + L.tile_expert);
   int* slot = reinterpret_cast<int*>(ws + L.slot);
@@ -180,9 +187,9 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   __half* hp = reinterpret_cast<__half*>(ws + L.hp);
   __half* yp = reinterpret_cast<__half*>(ws + L.yp);
   const int d = c.hidden, I = c.intermediate, E = c.experts, K = c.top_k;
-  cudaError_t e = cudaMemsetAsync(counts, 0, kMoeMaxExperts * sizeof(int), st);
+  cudaError_t e = cudaSuccess;
   // router logits
-  if (e == cudaSuccess) {
+  {
     GemmCore core;
     core_init(core, T, E, 64, 64, h->status);
     if (!map2d(&core.maps[0], x, true, d, T, d, 128)) return MOT_ERR_CUDA;
@@ -197,16 +204,16 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   }
   const int warps_grid = std::max(1, std::min((T + 7) / 8, 16 * h->num_sms));
   if (e == cudaSuccess)
-    e = launch_pdl(moe_route_kernel, dim3(warps_grid), dim3(256), 0, st, static_cast<const float*>(logits), T, E, K,
-                   idx, wts, counts);
+    e = launch_pdl(moe_route_kernel, dim3(L.nblk), dim3(kMoeRouteWarps * 32), 0, st,
+                   static_cast<const float*>(logits), T, E, K, idx, wts, pos, blk_cnt);
   if (e == cudaSuccess)
-    e = launch_pdl(moe_offsets_kernel, dim3(1), dim3(256), 0, st, static_cast<const int*>(counts), E, L.tiles, offsets,
-                   tile_expert, total_rows, fill);
-  const int disp_grid = std::max(1, std::min((T + 7) / 8, 16 * h->num_sms));
+    e = launch_pdl(moe_offsets_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int*>(blk_cnt), L.nblk, E,
+                   L.tiles, blk_base, counts, offsets, tile_expert, total_rows);
   if (e == cudaSuccess)
-    e = launch_pdl(moe_dispatch_kernel, dim3(disp_grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), T, K,
-                   d, static_cast<const int*>(idx), static_cast<const int*>(offsets), static_cast<const int*>(counts),
-                   fill, static_cast<const int*>(tile_expert), static_cast<const int*>(total_rows), xp, slot);
+    e = launch_pdl(moe_dispatch_kernel, dim3(warps_grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), T,
+                   K, E, d, L.nblk, static_cast<const int*>(idx), static_cast<const int*>(pos),
+                   static_cast<const int*>(blk_base), static_cast<const int*>(offsets),
+                   static_cast<const int*>(counts), xp, slot);
   // gate/up of every slot's expert, SwiGLU -> h (f16)
   if (e == cudaSuccess) {
     GemmCore core;
