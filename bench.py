@@ -450,6 +450,8 @@ def mlp_steps(dev, flush, stream, args, world):
         dp.barrier(world)
         steps = max(3, args.steps // 2)
         f_ms, b_ms = [], []
+        clk = ClockSampler(dev.index if dev.index is not None else 0)
+        clk.start()
         for _ in range(steps):
             flush.zero_()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
@@ -458,6 +460,7 @@ def mlp_steps(dev, flush, stream, args, world):
             f_ms.append(ev[0].elapsed_time(ev[1]))
             if train:
                 b_ms.append(ev[1].elapsed_time(ev[2]))
+        clocks = clk.stop()
         stages = {}
         mot_dev_mlp_profile(m.handle, True)
         for _ in range(steps):
@@ -478,7 +481,7 @@ def mlp_steps(dev, flush, stream, args, world):
                "fwd_ms": f, "fwd_tflops": fl / (f / 1e3) / 1e12,
                "fwd_frac_of_bf16_peak": fl / (f / 1e3) / 1e12 / peaks["bf16_tflops"],
                "tokens_per_s": world * wl.tokens / (f / 1e3),
-               "stages_ms": {n: sum(v) / steps for n, v in stages.items()}}
+               "stages_ms": {n: sum(v) / steps for n, v in stages.items()}, "clocks": clocks}
         if train:
             b = dp.max_over_ranks(statistics.mean(b_ms), world, dev)
             bfl = 6.0 * wl.tokens * wl.hidden * wl.inter + 2.0 * wl.tokens * wl.lora_rank * 4 * (wl.hidden + wl.inter)
@@ -620,6 +623,8 @@ def moe_bench(dev, flush, stream, args, world):
     torch.cuda.synchronize(dev)
     dp.barrier(world)
     ms = []
+    clk = ClockSampler(dev.index if dev.index is not None else 0)
+    clk.start()
     for _ in range(max(3, args.steps // 2)):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -628,6 +633,7 @@ def moe_bench(dev, flush, stream, args, world):
         e1.record(stream)
         e1.synchronize()
         ms.append(e0.elapsed_time(e1))
+    clocks = clk.stop()
     assert moe.device_status() == 0
     moe.close()
     t = dp.max_over_ranks(statistics.mean(ms), world, dev)
@@ -635,7 +641,7 @@ def moe_bench(dev, flush, stream, args, world):
     peaks, _ = load_peaks()
     return {"workload": "moe_a3b_2048sq_cfg2_tokens", "tokens": T, "hidden": d, "experts": E, "top_k": K,
             "intermediate": I, "ms": t, "tokens_per_s": world * T / (t / 1e3), "tflops": fl / (t / 1e3) / 1e12,
-            "frac_of_bf16_peak": fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"]}
+            "frac_of_bf16_peak": fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], "clocks": clocks}
 
 
 def sustained_steps(bundle, dev, stream, args, world, local):
@@ -784,14 +790,16 @@ def run_ours(args):
         dp.barrier(world)
         torch.cuda.synchronize(dev)
         u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        uclk = ClockSampler(local)
+        uclk.start()
         u0.record(stream)
         for _ in range(k):
             layer.forward(x_u, kc_u, vc_u, pl_u, y=y_u, workspace=ws_u)
         u1.record(stream)
         u1.synchronize()
-        return dp.max_over_ranks(u0.elapsed_time(u1) / k, world, dev)
+        return dp.max_over_ranks(u0.elapsed_time(u1) / k, world, dev), uclk.stop()
 
-    unflushed = unflushed_ms(args.steps)
+    unflushed, unflushed_clocks = unflushed_ms(args.steps)
 
     # end to end through the public call with host buffers. Every step copies
     # its inputs (x and the prefix cache) in from pinned host memory and its
@@ -974,7 +982,7 @@ def run_ours(args):
             "moe": moe,
             "sustained": sustained,
             "unflushed": {"ms_per_step": unflushed, "value": dp.aggregate_rate(tokens, 1, unflushed, world),
-                          "note": "same steps back to back, L2 not flushed"},
+                          "note": "same steps back to back, L2 not flushed", "clocks": unflushed_clocks},
         }
         print(json.dumps(line), flush=True)
     layer.close()

@@ -87,15 +87,14 @@ __global__ void __launch_bounds__(kMoeRouteWarps * 32) moe_route_kernel(
 // expert-major like blk_cnt) and the total count; then the expert block
 // offsets (each count padded to a multiple of 256), the M-tile table of the
 // grouped GEMMs (expert of each 256-row tile, -1 past the used rows, for all
-// `tiles` entries) and the total row count. One block of 32 warps, warp e
+// `tiles` entries). One block of 32 warps, warp e
 // scanning expert e: lane l sums a contiguous chunk of blocks (independent
 // loads), the lanes' sums are scanned by shuffles, and each lane writes its
 // chunk's running bases.
 __global__ void __launch_bounds__(1024) moe_offsets_kernel(const int* __restrict__ blk_cnt, int nblk, int E,
                                                            int tiles, int* __restrict__ blk_base,
                                                            int* __restrict__ counts, int* __restrict__ offsets,
-                                                           int* __restrict__ tile_expert,
-                                                           int* __restrict__ total_rows) {
+                                                           int* __restrict__ tile_expert) {
   grid_dep_launch();
   grid_dep_wait();
   __shared__ int cnt[kMoeMaxExperts];
@@ -133,7 +132,6 @@ __global__ void __launch_bounds__(1024) moe_offsets_kernel(const int* __restrict
       o += (cnt[j] + kMoeTileRows - 1) / kMoeTileRows * kMoeTileRows;
     }
     off[E] = o;
-    *total_rows = o;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < tiles; i += blockDim.x) {

@@ -54,7 +54,7 @@ MoeLayout make_moe_layout(const mot_moe_config& c, int T) {
   L.pos = take(t * K * 4);
   L.blk_cnt = take(static_cast<size_t>(L.nblk) * E * 4);
   L.blk_base = take(static_cast<size_t>(L.nblk) * E * 4);
-  L.small = take(3 * kMoeMaxExperts * 4);  // counts, offsets, total rows
+  L.small = take(2 * kMoeMaxExperts * 4);  // counts, offsets
   L.tile_expert = take(static_cast<size_t>(L.tiles) * 4);
   L.slot = take(t * K * 4);
   L.xp = take(static_cast<size_t>(L.rows) * d * 2);
@@ -180,7 +180,6 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
   int* blk_base = reinterpret_cast<int*>(ws + L.blk_base);
   int* counts = reinterpret_cast<int*>(ws + L.small);
   int* offsets = counts + kMoeMaxExperts;
-  int* total_rows = offsets + kMoeMaxExperts;
   int* tile_expert = reinterpret_cast<int*>(ws + L.tile_expert);
   int* slot = reinterpret_cast<int*>(ws + L.slot);
   __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(ws + L.xp);
@@ -208,7 +207,7 @@ mot_status mot_moe_forward(mot_moe_t h, const void* x, int32_t T, void* y, float
                    static_cast<const float*>(logits), T, E, K, idx, wts, pos, blk_cnt);
   if (e == cudaSuccess)
     e = launch_pdl(moe_offsets_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int*>(blk_cnt), L.nblk, E,
-                   L.tiles, blk_base, counts, offsets, tile_expert, total_rows);
+                   L.tiles, blk_base, counts, offsets, tile_expert);
   if (e == cudaSuccess)
     e = launch_pdl(moe_dispatch_kernel, dim3(warps_grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), T,
                    K, E, d, L.nblk, static_cast<const int*>(idx), static_cast<const int*>(pos),
