@@ -8,10 +8,11 @@
 // expert e occupy rows [offset[e], offset[e] + count[e]) of the permuted
 // buffers, each expert's block padded with zero rows to a multiple of 256
 // (one M tile of the pair GEMM), so an M tile never spans two experts.
-// Slots are assigned without global atomics: the routing kernel takes one
-// block per 64 tokens and numbers each expert's selections within the block
-// (shared-memory counters), a scan over the blocks gives every block's base
-// within each expert, and dispatch adds the two.
+// Slots are assigned in token order, without atomics: the routing kernel
+// takes one block per 64 tokens and numbers each expert's selections within
+// the block, a scan over the blocks gives every block's base within each
+// expert, and dispatch adds the two; the slot layout is the same on every
+// run.
 #pragma once
 
 #include "ptx.cuh"
@@ -33,25 +34,29 @@ constexpr int kMoeRouteTokens = kMoeRouteWarps * kMoeRouteTokensPerWarp;  // tok
 // (how many experts have a larger logit, or an equal one at a lower index:
 // the order of the probabilities, which exp keeps), so the selection has no
 // dependent rounds; the lanes ranked below top_k write their slot. Every
-// selection is numbered within its block and expert (topk_pos); blk_cnt[e][b]
-// is the block's count.
+// selection gets its number within its block and expert in token order
+// (topk_pos): lane e keeps a bit per token of its warp that chose expert e,
+// the warps' counts are scanned in shared memory, and the number is the
+// warp's base plus the bits below the token's. blk_cnt[e][b] is the block's
+// count.
 __global__ void __launch_bounds__(kMoeRouteWarps * 32) moe_route_kernel(
     const float* __restrict__ logits, int T, int E, int K, int* __restrict__ topk_idx, float* __restrict__ topk_w,
     int* __restrict__ topk_pos, int* __restrict__ blk_cnt) {
-  __shared__ int block_counts[kMoeMaxExperts];
-  if (threadIdx.x < kMoeMaxExperts) block_counts[threadIdx.x] = 0;
-  __syncthreads();
+  __shared__ int warp_counts[kMoeRouteWarps][kMoeMaxExperts];
   grid_dep_launch();
   grid_dep_wait();
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool live = lane < E;
-  const int t0 = blockIdx.x * kMoeRouteTokens + (threadIdx.x >> 5) * kMoeRouteTokensPerWarp;
+  const int t0 = blockIdx.x * kMoeRouteTokens + warp * kMoeRouteTokensPerWarp;
   float vv[kMoeRouteTokensPerWarp];
 #pragma unroll
   for (int i = 0; i < kMoeRouteTokensPerWarp; ++i)
     vv[i] = (live && t0 + i < T) ? logits[static_cast<long long>(t0 + i) * E + lane] : -INFINITY;
+  unsigned chosen = 0u;  // bit i: token t0 + i chose this lane's expert
+  int rank_of[kMoeRouteTokensPerWarp];
 #pragma unroll
   for (int i = 0; i < kMoeRouteTokensPerWarp; ++i) {
+    rank_of[i] = 0;
     const int t = t0 + i;
     if (t >= T) break;
     const float v = vv[i];
@@ -76,11 +81,23 @@ __global__ void __launch_bounds__(kMoeRouteWarps * 32) moe_route_kernel(
       const long long pr = static_cast<long long>(t) * K + rank;
       topk_idx[pr] = lane;
       topk_w[pr] = p / ws;
-      topk_pos[pr] = atomicAdd(&block_counts[lane], 1);
+      chosen |= 1u << i;
+      rank_of[i] = rank;
     }
   }
+  warp_counts[warp][lane] = __popc(chosen);
   __syncthreads();
-  if (threadIdx.x < E) blk_cnt[static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x] = block_counts[threadIdx.x];
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_counts[w][lane];
+#pragma unroll
+  for (int i = 0; i < kMoeRouteTokensPerWarp; ++i)
+    if (chosen & (1u << i))
+      topk_pos[static_cast<long long>(t0 + i) * K + rank_of[i]] = base + __popc(chosen & ((1u << i) - 1u));
+  if (threadIdx.x < E) {
+    int total = 0;
+    for (int w = 0; w < kMoeRouteWarps; ++w) total += warp_counts[w][threadIdx.x];
+    blk_cnt[static_cast<long long>(threadIdx.x) * gridDim.x + blockIdx.x] = total;
+  }
 }
 
 // Per expert: the exclusive scan of the routing blocks' counts (blk_base,

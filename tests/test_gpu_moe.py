@@ -78,8 +78,9 @@ def test_moe_a3b_dims_1024sq_cfg_tokens(cuda_ready):
     moe, td, y, y32, ex = _run(t, synth.MOE_TOP_K)
     frac_clear = _check(t, synth.MOE_TOP_K, y, y32, ex)
     assert frac_clear > 0.99
-    # deterministic although slots are assigned by atomics: every row of an
-    # expert's GEMM is computed on its own and the combine sums in rank order
+    # deterministic: the slots of an expert are in token order, every row of
+    # an expert's GEMM is computed on its own and the combine sums in rank
+    # order
     y32b = torch.empty_like(y32)
     moe.forward(td["x"], y_f32=y32b)
     torch.cuda.synchronize()
