@@ -1069,14 +1069,24 @@ struct EpiQkv {
           }
           p.rstd[static_cast<long long>(m) * (p.Hq + p.Hkv) + head] = rs;
         }
-        const float2* cs = p.rope + static_cast<long long>(pos) * 64;
+        // (cos, sin) of two pairs and four gains per 16-byte load (the table
+        // rows and the gains are 16-byte aligned)
+        const float4* cs4 = reinterpret_cast<const float4*>(p.rope + static_cast<long long>(pos) * 64);
+        const float4* g4 = reinterpret_cast<const float4*>(gamma);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float2 t = __ldg(cs + j);
-          const float a = v[j] * rs * __ldg(gamma + j);
-          const float c = v[j + 64] * rs * __ldg(gamma + j + 64);
-          v[j] = a * t.x - c * t.y;
-          v[j + 64] = c * t.x + a * t.y;
+        for (int j4 = 0; j4 < 16; ++j4) {
+          const float4 t01 = __ldg(cs4 + 2 * j4), t23 = __ldg(cs4 + 2 * j4 + 1);
+          const float4 ga = __ldg(g4 + j4), gc = __ldg(g4 + 16 + j4);
+          const float tc[4] = {t01.x, t01.z, t23.x, t23.z}, ts[4] = {t01.y, t01.w, t23.y, t23.w};
+          const float gl[4] = {ga.x, ga.y, ga.z, ga.w}, gh[4] = {gc.x, gc.y, gc.z, gc.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 4 * j4 + u;
+            const float a = v[j] * rs * gl[u];
+            const float c = v[j + 64] * rs * gh[u];
+            v[j] = a * tc[u] - c * ts[u];
+            v[j + 64] = c * tc[u] + a * ts[u];
+          }
         }
         dst = is_q ? p.q_out + (static_cast<long long>(b * p.Hq + head) * p.N + n) * 128
                    : p.k_out + (static_cast<long long>(b * p.Hkv + head - p.Hq) * p.Lcap + pos) * 128;
