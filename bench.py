@@ -870,10 +870,12 @@ def run_ours(args):
     also = None
     if not args.skip_also:
         wl1, _, td1, layer1 = make(ALSO_INDEX)
-        ms1, _, _ = device_steps(wl1, td1, layer1, max(3, args.steps // 2), args.warmup, False)
+        ms1, st1, _ = device_steps(wl1, td1, layer1, max(3, args.steps // 2), args.warmup, True)
         max1 = dp.max_over_ranks(sum(ms1), world, dev)
+        fl1 = sum(stage_work(wl1, n)[0] for n in st1)
         also = {"workload": wl1.name, "value": dp.aggregate_rate(wl1.batch * wl1.img_tokens, len(ms1), max1, world),
-                "ms_per_step": max1 / len(ms1)}
+                "ms_per_step": max1 / len(ms1), "tflops": fl1 / (max1 / len(ms1) / 1e3) / 1e12,
+                "stages_ms": {n: sum(v) / len(ms1) for n, v in st1.items()}}
         layer1.close()
         # the edit workload: adapters baked into the base (merge at load), then rank-0 calls
         wl3, _, td3, layer3 = make(EDIT_INDEX)
