@@ -27,6 +27,21 @@ def _ptr(t: Optional[torch.Tensor]):
     return c_void_p(t.data_ptr())
 
 
+_BF16, _F32, _I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+def _dptr(t: Optional[torch.Tensor], dtype: Optional[torch.dtype] = None, name: str = "tensor"):
+    """Pointer of a device argument: a contiguous CUDA tensor (of `dtype`
+    when given). A host tensor here would hand the kernels a host address."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    return _ptr(t)
+
+
 def _stream(stream) -> c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -48,7 +63,7 @@ def mot_attn_query_sizes(cfg: MotAttnConfig, batch: int, img_tokens: int, prefix
 
 
 def mot_attn_create(cfg: MotAttnConfig, weights: Dict[str, torch.Tensor], stream=None) -> c_void_p:
-    w = MotAttnWeights(*[_ptr(weights.get(n)) for n in WEIGHT_NAMES])
+    w = MotAttnWeights(*[_dptr(weights.get(n), _BF16, n) for n in WEIGHT_NAMES])
     h = c_void_p()
     check(lib().mot_attn_create(byref(cfg), byref(w), _stream(stream), byref(h)), "mot_attn_create")
     return h
@@ -57,9 +72,11 @@ def mot_attn_create(cfg: MotAttnConfig, weights: Dict[str, torch.Tensor], stream
 def mot_attn_forward(h, x, batch, img_tokens, k_cache, v_cache, prefix_len: Sequence[int], prefix_max, y,
                      y_f32=None, saved=None, workspace=None, stream=None) -> None:
     pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
-    check(lib().mot_attn_forward(h, _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl, prefix_max,
-                                 _ptr(y), _ptr(y_f32), _ptr(saved), saved.numel() if saved is not None else 0,
-                                 _ptr(workspace), workspace.numel() if workspace is not None else 0,
+    check(lib().mot_attn_forward(h, _dptr(x, _BF16, "x"), batch, img_tokens, _dptr(k_cache, _BF16, "k_cache"),
+                                 _dptr(v_cache, _BF16, "v_cache"), pl, prefix_max, _dptr(y, _BF16, "y"),
+                                 _dptr(y_f32, _F32, "y_f32"), _dptr(saved, None, "saved"),
+                                 saved.numel() if saved is not None else 0, _dptr(workspace, None, "workspace"),
+                                 workspace.numel() if workspace is not None else 0,
                                  _stream(stream)), "mot_attn_forward")
 
 
@@ -68,8 +85,9 @@ def mot_attn_prefix_forward(h, x, batch, tokens, lengths: Sequence[int], y, k_ca
     """The prefix tower's layer over the prompt (causal), writing the layer's
     bf16 cache entry; see include/mot_attn.h."""
     ln = (c_int32 * batch)(*[int(v) for v in lengths])
-    check(lib().mot_attn_prefix_forward(h, _ptr(x), batch, tokens, ln, _ptr(y), _ptr(y_f32), _ptr(k_cache_out),
-                                        _ptr(v_cache_out), _ptr(workspace),
+    check(lib().mot_attn_prefix_forward(h, _dptr(x, _BF16, "x"), batch, tokens, ln, _dptr(y, _BF16, "y"),
+                                        _dptr(y_f32, _F32, "y_f32"), _dptr(k_cache_out, _BF16, "k_cache_out"),
+                                        _dptr(v_cache_out, _BF16, "v_cache_out"), _dptr(workspace, None, "workspace"),
                                         workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_attn_prefix_forward")
 
@@ -79,8 +97,10 @@ def mot_attn_forward_noalloc(h, x, batch, img_tokens, k_cache, v_cache, prefix_l
     """Forward whose scratch is the library's own fixed device array (no
     workspace argument, no allocation); see include/mot_attn.h."""
     pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
-    check(lib().mot_attn_forward_noalloc(h, _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl,
-                                         prefix_max, _ptr(y), _ptr(y_f32), _stream(stream)),
+    check(lib().mot_attn_forward_noalloc(h, _dptr(x, _BF16, "x"), batch, img_tokens,
+                                         _dptr(k_cache, _BF16, "k_cache"), _dptr(v_cache, _BF16, "v_cache"), pl,
+                                         prefix_max, _dptr(y, _BF16, "y"), _dptr(y_f32, _F32, "y_f32"),
+                                         _stream(stream)),
           "mot_attn_forward_noalloc")
 
 
@@ -88,11 +108,13 @@ def mot_attn_backward(h, dy, x, batch, img_tokens, k_cache, v_cache, prefix_len:
                       saved, dx, dx_f32=None, d_a=None, d_b=None, accumulate=False, workspace=None,
                       stream=None) -> None:
     pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
-    da = (c_void_p * 4)(*[_ptr(t) for t in (d_a or [None] * 4)])
-    db = (c_void_p * 4)(*[_ptr(t) for t in (d_b or [None] * 4)])
-    check(lib().mot_attn_backward(h, _ptr(dy), _ptr(x), batch, img_tokens, _ptr(k_cache), _ptr(v_cache), pl,
-                                  prefix_max, _ptr(saved), saved.numel() if saved is not None else 0, _ptr(dx),
-                                  _ptr(dx_f32), da, db, int(bool(accumulate)), _ptr(workspace),
+    da = (c_void_p * 4)(*[_dptr(t, _F32, "d_a") for t in (d_a or [None] * 4)])
+    db = (c_void_p * 4)(*[_dptr(t, _F32, "d_b") for t in (d_b or [None] * 4)])
+    check(lib().mot_attn_backward(h, _dptr(dy, _BF16, "dy"), _dptr(x, _BF16, "x"), batch, img_tokens,
+                                  _dptr(k_cache, _BF16, "k_cache"), _dptr(v_cache, _BF16, "v_cache"), pl,
+                                  prefix_max, _dptr(saved, None, "saved"), saved.numel() if saved is not None else 0,
+                                  _dptr(dx, _BF16, "dx"), _dptr(dx_f32, _F32, "dx_f32"), da, db,
+                                  int(bool(accumulate)), _dptr(workspace, None, "workspace"),
                                   workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_attn_backward")
 
@@ -121,12 +143,14 @@ def mot_attn_forward_host(h, xs, batch, img_tokens, k_caches, v_caches, prefix_l
     kc = _host_ptrs(k_caches) if k_caches is not None else None
     vc = _host_ptrs(v_caches) if v_caches is not None else None
     check(lib().mot_attn_forward_host(h, steps, _host_ptrs(xs), batch, img_tokens, kc, vc, pl, prefix_max,
-                                      _host_ptrs(ys), _ptr(staging), staging.numel(), _ptr(workspace),
+                                      _host_ptrs(ys), _dptr(staging, None, "staging"), staging.numel(),
+                                      _dptr(workspace, None, "workspace"),
                                       workspace.numel(), _stream(stream)), "mot_attn_forward_host")
 
 
 def mot_attn_merge_lora(h, w_q_out, w_k_out, w_v_out, w_o_out, stream=None) -> None:
-    check(lib().mot_attn_merge_lora(h, _ptr(w_q_out), _ptr(w_k_out), _ptr(w_v_out), _ptr(w_o_out),
+    check(lib().mot_attn_merge_lora(h, _dptr(w_q_out, _BF16, "w_q_out"), _dptr(w_k_out, _BF16, "w_k_out"),
+                                    _dptr(w_v_out, _BF16, "w_v_out"), _dptr(w_o_out, _BF16, "w_o_out"),
                                     _stream(stream)), "mot_attn_merge_lora")
 
 

@@ -14,7 +14,7 @@ from typing import Dict, Optional, Tuple
 import torch
 
 from ._abi import MotMlpConfig, MotMlpWeights, check, lib
-from .layer import _ptr, _stream
+from .layer import _BF16, _F32, _dptr, _stream
 
 MLP_WEIGHT_NAMES = ("w_gate", "w_up", "w_down", "a_gate", "a_up", "a_down", "b_gate", "b_up", "b_down")
 
@@ -31,25 +31,27 @@ def mot_mlp_query_sizes(cfg: MotMlpConfig, tokens: int) -> Tuple[int, int]:
 
 
 def mot_mlp_create(cfg: MotMlpConfig, weights: Dict[str, torch.Tensor], stream=None) -> c_void_p:
-    w = MotMlpWeights(*[_ptr(weights.get(n)) for n in MLP_WEIGHT_NAMES])
+    w = MotMlpWeights(*[_dptr(weights.get(n), _BF16, n) for n in MLP_WEIGHT_NAMES])
     h = c_void_p()
     check(lib().mot_mlp_create(byref(cfg), byref(w), _stream(stream), byref(h)), "mot_mlp_create")
     return h
 
 
 def mot_mlp_forward(h, x, tokens, y, y_f32=None, saved=None, workspace=None, stream=None) -> None:
-    check(lib().mot_mlp_forward(h, _ptr(x), tokens, _ptr(y), _ptr(y_f32), _ptr(saved),
-                                saved.numel() if saved is not None else 0, _ptr(workspace),
+    check(lib().mot_mlp_forward(h, _dptr(x, _BF16, "x"), tokens, _dptr(y, _BF16, "y"), _dptr(y_f32, _F32, "y_f32"),
+                                _dptr(saved, None, "saved"), saved.numel() if saved is not None else 0,
+                                _dptr(workspace, None, "workspace"),
                                 workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_mlp_forward")
 
 
 def mot_mlp_backward(h, dy, x, tokens, saved, dx, dx_f32=None, d_a=None, d_b=None, accumulate=False,
                      workspace=None, stream=None) -> None:
-    da = (c_void_p * 3)(*[_ptr(t) for t in (d_a or [None] * 3)])
-    db = (c_void_p * 3)(*[_ptr(t) for t in (d_b or [None] * 3)])
-    check(lib().mot_mlp_backward(h, _ptr(dy), _ptr(x), tokens, _ptr(saved), saved.numel(), _ptr(dx), _ptr(dx_f32),
-                                 da, db, int(bool(accumulate)), _ptr(workspace),
+    da = (c_void_p * 3)(*[_dptr(t, _F32, "d_a") for t in (d_a or [None] * 3)])
+    db = (c_void_p * 3)(*[_dptr(t, _F32, "d_b") for t in (d_b or [None] * 3)])
+    check(lib().mot_mlp_backward(h, _dptr(dy, _BF16, "dy"), _dptr(x, _BF16, "x"), tokens, _dptr(saved, None, "saved"),
+                                 saved.numel(), _dptr(dx, _BF16, "dx"), _dptr(dx_f32, _F32, "dx_f32"),
+                                 da, db, int(bool(accumulate)), _dptr(workspace, None, "workspace"),
                                  workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_mlp_backward")
 

@@ -9,7 +9,7 @@ from typing import Dict
 import torch
 
 from ._abi import MotMoeConfig, MotMoeWeights, check, lib
-from .layer import _ptr, _stream
+from .layer import _BF16, _F32, _I32, _dptr, _stream
 
 
 def mot_moe_query_workspace(cfg: MotMoeConfig, tokens: int) -> int:
@@ -19,14 +19,15 @@ def mot_moe_query_workspace(cfg: MotMoeConfig, tokens: int) -> int:
 
 
 def mot_moe_create(cfg: MotMoeConfig, weights: Dict[str, torch.Tensor], stream=None) -> c_void_p:
-    w = MotMoeWeights(*[_ptr(weights[n]) for n in ("w_router", "w_gate", "w_up", "w_down")])
+    w = MotMoeWeights(*[_dptr(weights[n], _BF16, n) for n in ("w_router", "w_gate", "w_up", "w_down")])
     h = c_void_p()
     check(lib().mot_moe_create(byref(cfg), byref(w), _stream(stream), byref(h)), "mot_moe_create")
     return h
 
 
 def mot_moe_forward(h, x, tokens, y, y_f32=None, experts_out=None, workspace=None, stream=None) -> None:
-    check(lib().mot_moe_forward(h, _ptr(x), tokens, _ptr(y), _ptr(y_f32), _ptr(experts_out), _ptr(workspace),
+    check(lib().mot_moe_forward(h, _dptr(x, _BF16, "x"), tokens, _dptr(y, _BF16, "y"), _dptr(y_f32, _F32, "y_f32"),
+                                _dptr(experts_out, _I32, "experts_out"), _dptr(workspace, None, "workspace"),
                                 workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_moe_forward")
 

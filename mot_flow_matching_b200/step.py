@@ -12,15 +12,16 @@ from typing import Sequence
 import torch
 
 from ._abi import MotStepConfig, MotStepModel, check, lib
-from .layer import _ptr, _stream
+from .layer import _BF16, _F32, _dptr, _stream
 
 
 def mot_step_create(cfg: MotStepConfig, attn_handles, mlp_handles, norm_in, norm_post, w_in, norm_out, w_out,
                     stream=None) -> c_void_p:
     n = cfg.n_layers
     arr = lambda xs: (c_void_p * n)(*[x.value if isinstance(x, c_void_p) else x for x in xs])
-    model = MotStepModel(arr(attn_handles), arr(mlp_handles), arr([_ptr(t) for t in norm_in]),
-                         arr([_ptr(t) for t in norm_post]), _ptr(w_in), _ptr(norm_out), _ptr(w_out))
+    model = MotStepModel(arr(attn_handles), arr(mlp_handles), arr([_dptr(t, _BF16, "norm_in") for t in norm_in]),
+                         arr([_dptr(t, _BF16, "norm_post") for t in norm_post]), _dptr(w_in, _BF16, "w_in"),
+                         _dptr(norm_out, _BF16, "norm_out"), _dptr(w_out, _BF16, "w_out"))
     h = c_void_p()
     check(lib().mot_step_create(byref(cfg), byref(model), _stream(stream), byref(h)), "mot_step_create")
     return h
@@ -36,12 +37,13 @@ def mot_step_forward(h, z, batch, img_tokens, k_caches, v_caches, prefix_len: Se
                      sigma_next, cfg_scale, img_cfg_scale, t_eps, z_next, z_next_bf16=None, workspace=None,
                      stream=None) -> None:
     n = len(k_caches)
-    kc = (c_void_p * n)(*[_ptr(t) for t in k_caches])
-    vc = (c_void_p * n)(*[_ptr(t) for t in v_caches])
+    kc = (c_void_p * n)(*[_dptr(t, _BF16, "k_cache") for t in k_caches])
+    vc = (c_void_p * n)(*[_dptr(t, _BF16, "v_cache") for t in v_caches])
     pl = (c_int32 * batch)(*[int(v) for v in prefix_len])
-    check(lib().mot_step_forward(h, _ptr(z), batch, img_tokens, kc, vc, pl, prefix_max, float(sigma),
+    check(lib().mot_step_forward(h, _dptr(z, _F32, "z"), batch, img_tokens, kc, vc, pl, prefix_max, float(sigma),
                                  float(sigma_next), float(cfg_scale), float(img_cfg_scale), float(t_eps),
-                                 _ptr(z_next), _ptr(z_next_bf16), _ptr(workspace),
+                                 _dptr(z_next, _F32, "z_next"), _dptr(z_next_bf16, _BF16, "z_next_bf16"),
+                                 _dptr(workspace, None, "workspace"),
                                  workspace.numel() if workspace is not None else 0, _stream(stream)),
           "mot_step_forward")
 

@@ -140,3 +140,20 @@ def test_step_create_rejects_bad_arguments_before_cuda(L):
                 _abi.MotStepConfig(n_layers=1, hidden=4096, patch_dim=3072, rms_eps=-1.0)):
         assert L.mot_step_create(byref(bad), byref(model), None, byref(out)) == _abi.MOT_ERR_INVALID_ARGUMENT
     assert L.mot_step_create(byref(cfg), None, None, byref(out)) == _abi.MOT_ERR_INVALID_ARGUMENT
+
+
+def test_bindings_refuse_host_tensors_and_wrong_dtypes():
+    # a host tensor where the C call takes a device pointer would hand the
+    # kernels a host address: refused in the binding, before the call
+    import torch
+    from mot_flow_matching_b200.layer import _dptr, mot_attn_forward
+    from mot_flow_matching_b200.moe import mot_moe_forward
+    with pytest.raises(ValueError, match="CUDA"):
+        _dptr(torch.zeros(4, dtype=torch.bfloat16), torch.bfloat16, "x")
+    with pytest.raises(ValueError, match="CUDA"):
+        mot_attn_forward(c_void_p(1), torch.zeros(1, 16, 512, dtype=torch.bfloat16), 1, 16, None, None, [0], 0,
+                         torch.zeros(1, 16, 512, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        mot_moe_forward(c_void_p(1), torch.zeros(4, 256, dtype=torch.bfloat16), 4,
+                        torch.zeros(4, 256, dtype=torch.bfloat16))
+    assert _dptr(None, torch.float32) is None
