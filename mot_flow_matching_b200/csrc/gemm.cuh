@@ -635,6 +635,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------------ epilogues
+// 64 bytes of one row: two whole 32-byte sectors when the address allows,
+// else four 16-byte stores (outputs are only required to be 16-byte aligned)
+__device__ __forceinline__ void store_row64(void* dst, const uint32_t (&w)[16]) {
+  if ((reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
+    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_v8(static_cast<uint8_t*>(dst) + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+  } else {
+    uint4* d = static_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
 __device__ __forceinline__ void load_row32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   tmem_ld32(taddr, r);
@@ -742,15 +755,7 @@ struct EpiStore {
       if constexpr (!kBf16) amax = fmax3_nan(amax, fabsf(a), fabsf(b));
       w[k] = pack2<kBf16>(a, b);
     }
-    if ((reinterpret_cast<uintptr_t>(row) & 31) == 0) {
-      // two whole 32-byte sectors per thread instead of four half sectors
-      st_global_v8(row, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-      st_global_v8(row + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
-    } else {
-      uint4* dst = reinterpret_cast<uint4*>(row);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-    }
+    store_row64(row, w);
   }
   template <int BN>
   __device__ __forceinline__ static void apply(const Params& p, uint32_t taddr, int m0, int n0, int row,
@@ -1075,39 +1080,35 @@ struct EpiQkv {
           }
           p.rstd[static_cast<long long>(m) * (p.Hq + p.Hkv) + head] = rs;
         }
-        // (cos, sin) of two pairs and four gains per 16-byte load (the table
-        // rows and the gains are 16-byte aligned)
-        const float4* cs4 = reinterpret_cast<const float4*>(p.rope + static_cast<long long>(pos) * 64);
-        const float4* g4 = reinterpret_cast<const float4*>(gamma);
+        const float2* cs = p.rope + static_cast<long long>(pos) * 64;
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-          const float4 t01 = __ldg(cs4 + 2 * j4), t23 = __ldg(cs4 + 2 * j4 + 1);
-          const float4 ga = __ldg(g4 + j4), gc = __ldg(g4 + 16 + j4);
-          const float tc[4] = {t01.x, t01.z, t23.x, t23.z}, ts[4] = {t01.y, t01.w, t23.y, t23.w};
-          const float gl[4] = {ga.x, ga.y, ga.z, ga.w}, gh[4] = {gc.x, gc.y, gc.z, gc.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = 4 * j4 + u;
-            const float a = v[j] * rs * gl[u];
-            const float c = v[j + 64] * rs * gh[u];
-            v[j] = a * tc[u] - c * ts[u];
-            v[j + 64] = c * tc[u] + a * ts[u];
-          }
+        for (int j = 0; j < 64; ++j) {
+          const float2 t = __ldg(cs + j);
+          const float a = v[j] * rs * __ldg(gamma + j);
+          const float c = v[j + 64] * rs * __ldg(gamma + j + 64);
+          v[j] = a * t.x - c * t.y;
+          v[j + 64] = c * t.x + a * t.y;
         }
         dst = is_q ? p.q_out + (static_cast<long long>(b * p.Hq + head) * p.N + n) * 128
                    : p.k_out + (static_cast<long long>(b * p.Hkv + head - p.Hq) * p.Lcap + pos) * 128;
       } else {
         dst = p.v_out + (static_cast<long long>(b * p.Hkv + head - p.Hq - p.Hkv) * p.Lcap + pos) * 128;
       }
-      uint4* d4 = reinterpret_cast<uint4*>(dst);
+      // 32 bytes at a time (few live registers beside the 128 values)
+      const bool a32 = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        uint4 w;
-        w.x = pack_half2(v[8 * i + 0], v[8 * i + 1]);
-        w.y = pack_half2(v[8 * i + 2], v[8 * i + 3]);
-        w.z = pack_half2(v[8 * i + 4], v[8 * i + 5]);
-        w.w = pack_half2(v[8 * i + 6], v[8 * i + 7]);
-        d4[i] = w;
+      for (int q = 0; q < 8; ++q) {
+        const float* e = v + 16 * q;
+        const uint32_t w0 = pack_half2(e[0], e[1]), w1 = pack_half2(e[2], e[3]), w2 = pack_half2(e[4], e[5]),
+                       w3 = pack_half2(e[6], e[7]), w4 = pack_half2(e[8], e[9]), w5 = pack_half2(e[10], e[11]),
+                       w6 = pack_half2(e[12], e[13]), w7 = pack_half2(e[14], e[15]);
+        if (a32) {
+          st_global_v8(dst + 16 * q, w0, w1, w2, w3, w4, w5, w6, w7);
+        } else {
+          uint4* d = reinterpret_cast<uint4*>(dst + 16 * q);
+          d[0] = make_uint4(w0, w1, w2, w3);
+          d[1] = make_uint4(w4, w5, w6, w7);
+        }
       }
       if (p.kc_out && head >= p.Hq) {
         const bool is_k = head < p.Hq + p.Hkv;
@@ -1171,26 +1172,18 @@ struct EpiSwiGLU {
         amax = fmax3_nan(amax, fabsf(h0), fabsf(h1));
         hw[k] = pack_half2(h0, h1);
       }
-      uint4* hd = reinterpret_cast<uint4*>(p.h + off);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) hd[q] = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+      store_row64(p.h + off, hw);
       if (p.g_out) {
-        uint4* gd = reinterpret_cast<uint4*>(p.g_out + off);
-        uint4* ud = reinterpret_cast<uint4*>(p.u_out + off);
+        uint32_t gw[16], uw[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t gw[4], uw[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = 8 * q + 2 * k;
-            amax = fmax3_nan(amax, fabsf(__uint_as_float(gr[e])), fabsf(__uint_as_float(gr[e + 1])));
-            amax = fmax3_nan(amax, fabsf(__uint_as_float(ur[e])), fabsf(__uint_as_float(ur[e + 1])));
-            gw[k] = pack_half2(__uint_as_float(gr[e]), __uint_as_float(gr[e + 1]));
-            uw[k] = pack_half2(__uint_as_float(ur[e]), __uint_as_float(ur[e + 1]));
-          }
-          gd[q] = make_uint4(gw[0], gw[1], gw[2], gw[3]);
-          ud[q] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+        for (int k = 0; k < 16; ++k) {
+          amax = fmax3_nan(amax, fabsf(__uint_as_float(gr[2 * k])), fabsf(__uint_as_float(gr[2 * k + 1])));
+          amax = fmax3_nan(amax, fabsf(__uint_as_float(ur[2 * k])), fabsf(__uint_as_float(ur[2 * k + 1])));
+          gw[k] = pack_half2(__uint_as_float(gr[2 * k]), __uint_as_float(gr[2 * k + 1]));
+          uw[k] = pack_half2(__uint_as_float(ur[2 * k]), __uint_as_float(ur[2 * k + 1]));
         }
+        store_row64(p.g_out + off, gw);
+        store_row64(p.u_out + off, uw);
       }
       overflow |= !(amax <= 65504.f);
     }
