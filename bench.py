@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     "attn_fwd": {"sha256": "f35c17d939924ee887ac497ea302c33107340a8f3b9650d1cb8c6f22c4442d80",
                  "bytes": 105389568 + 32933376},
-    "qkv_gemm": {"sha256": "33aaa982e0013e9285daab26c199a91efc6ee068ef654774d1ef08b070cfcae6",
-                 "bytes": 214257408 + 81502464},
+    "qkv_gemm": {"sha256": "0d41e561dca3ab88617e17057778f06f2ba99e11707cd22bdf0b5b1c8b2cb2a0",
+                 "bytes": 234373120 + 84449536},
 }
 KERNEL_SOURCES = {"attn_fwd": "attn_fwd.cuh", "qkv_gemm": "gemm.cuh", "o_gemm": "gemm.cuh"}
 
