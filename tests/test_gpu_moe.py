@@ -62,7 +62,9 @@ def _check(t, top_k, y, y32, ex):
     return clear.mean()
 
 
-@pytest.mark.parametrize("T,E,K", [(1, 8, 2), (77, 8, 8), (300, 16, 4), (513, 32, 8)])
+@pytest.mark.parametrize("T,E,K", [(1, 8, 2), (77, 8, 8), (300, 16, 4), (513, 32, 8),
+                                   (64, 4, 1),     # top-1, exactly one routing block of tokens
+                                   (130, 1, 1)])   # one expert: the dense SwiGLU MLP
 def test_moe_small_dims(cuda_ready, T, E, K):
     t = synth.make_moe_inputs(T, 256, 128, E, 8100 + T)
     t["w_router"] = (t["w_router"].float() * 8).to(torch.bfloat16)  # a spread of router probabilities

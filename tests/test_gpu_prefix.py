@@ -125,3 +125,28 @@ def test_prefix_cache_feeds_gen_forward_end_to_end(cuda_ready):
     assert_parity(y32.double().cpu().numpy(), ref["y"], "gen y f32 over the GPU-built cache")
     player.close()
     glayer.close()
+
+
+def test_prefix_forward_refuses_empty_and_overlong_prompts(cuda_ready):
+    # a branch with no prompt token (or more than N) has no causal key range:
+    # refused on the host before anything is launched; the handle stays usable
+    from mot_flow_matching_b200._abi import MOT_ERR_ALIGNMENT, MOT_ERR_INVALID_ARGUMENT, MotError
+    from mot_flow_matching_b200.layer import mot_attn_prefix_forward
+    wl, t = _prefix_inputs(2, 64, 5500, synth.LayerDims(**SMALL))
+    td = to_dev(t)
+    layer = make_layer(wl, td)
+    for lengths in ([0, 64], [64, 65], [64, -1]):
+        with pytest.raises(MotError) as e:
+            layer.prefix_forward(td["x"], lengths)
+        assert e.value.status == MOT_ERR_INVALID_ARGUMENT, lengths
+    y = torch.empty_like(td["x"])
+    kc = torch.empty(2 * 2 * 64 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(MotError) as e:  # cache output 2 bytes off the 16-byte alignment
+        mot_attn_prefix_forward(layer.handle, td["x"], 2, 64, [64, 64], y, kc[1:], kc[1:],
+                                workspace=layer.workspace(2, 64, 0))
+    assert e.value.status == MOT_ERR_ALIGNMENT
+    # still usable
+    y, kc2, vc2 = layer.prefix_forward(td["x"], [64, 10])
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    layer.close()
