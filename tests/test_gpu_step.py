@@ -142,18 +142,21 @@ def test_step_small_dims_x0(cuda_ready, B, N, P, plen, n_layers, rank, cfg, img_
     step.close()
 
 
-def test_step_euler_update(cuda_ready):
+@pytest.mark.parametrize("which", ["schedule_step", "below_t_eps"])
+def test_step_euler_update(cuda_ready, which):
     wl = synth.Workload("step", 2, 160, 48, 16, 16.0, dims=SMALL)
     inp = synth.make_step_inputs(2, wl, 384, 256, 7300)
     step, keep, _ = _build(inp, wl, 384)
     sig = SO.sigma_schedule(8, 3.0)
-    s0, s1 = float(sig[3]), float(sig[4])
+    # a step of the shifted schedule, or the last one from sigma = 0.01 below
+    # t_eps = 0.02, where the velocity divides by t_eps instead of sigma
+    s0, s1 = (float(sig[3]), float(sig[4])) if which == "schedule_step" else (0.01, 0.0)
     # cfg 1: the update applied to the conditional branch's x0 (the guidance
     # combine has its own test)
     got = _run(step, keep, inp, wl, [48, 48], s0, s1, 1.0, 1.0)
     ref = _oracle(inp, wl, [48, 48], s0, s1, 1.0, 1.0)
     z = inp["z"].double().numpy()
-    # the update part of the step, z_next - z = (s1 - s0) (z - x0) / s0
+    # the update part of the step, z_next - z = (s1 - s0) (z - x0) / max(s0, t_eps)
     assert_parity(got - z, ref["z_next"] - z, "z_next - z", **_bar(2))
     step.close()
 
