@@ -148,3 +148,16 @@ def test_backward_on_caller_stream(cuda_ready):
     assert layer.device_status(stream=s) == 0
     for got, ref in zip(host, [dx32_ref] + da_ref + db_ref):
         assert torch.equal(got.view(torch.int32), ref.cpu().view(torch.int32))
+
+
+@pytest.mark.parametrize("hidden,hq,hkv", [(512, 4, 4), (1024, 8, 2)])
+def test_backward_other_head_groupings(cuda_ready, hidden, hq, hkv):
+    # the dk/dv CTAs sum over the query heads of their KV head's group: group
+    # sizes 1 and 4 besides the small dims' 2
+    dims = synth.LayerDims(hidden=hidden, n_q_heads=hq, n_kv_heads=hkv)
+    wl = synth.Workload("groups", 2, 160, 48, 16, 32.0, train=True, dims=dims)
+    t = synth.make_inputs(wl, 9600 + hq * 10 + hkv, with_dy=True)
+    t["prefix_len"] = torch.tensor([48, 17], dtype=torch.int32)
+    dx, dx32, d_a, d_b, status, _ = run_backward(wl, t)
+    assert status == 0
+    check_all(wl, t, dx, dx32, d_a, d_b, oracle_backward(wl, t))

@@ -206,3 +206,23 @@ def test_f16_overflow_is_reported(cuda_ready):
     assert status == 7  # MOT_ERR_NUMERIC
     _, _, _, status = run_forward(layer, to_dev(synth.make_inputs(wl, 78, with_dy=False)))
     assert status == 0
+
+
+@pytest.mark.parametrize("hidden,hq,hkv", [
+    (512, 4, 4),     # no grouping: plain multi-head attention
+    (1024, 8, 2),    # a group of 4 query heads per KV head, as the full layer
+])
+def test_fwd_other_head_groupings(cuda_ready, hidden, hq, hkv):
+    # the KV head of query head h is h / (Hq / Hkv): other group sizes than
+    # the small dims' 2 and the full layer's 4-of-32
+    dims = synth.LayerDims(hidden=hidden, n_q_heads=hq, n_kv_heads=hkv)
+    wl = synth.Workload("groups", 2, 160, 48, 16, 32.0, dims=dims)
+    t = synth.make_inputs(wl, 9500 + hq * 10 + hkv, with_dy=False)
+    t["prefix_len"] = torch.tensor([48, 17], dtype=torch.int32)
+    td = to_dev(t)
+    layer = make_layer(wl, td)
+    y, y32, _, status = run_forward(layer, td)
+    assert status == 0
+    ref = oracle_forward(wl, t)
+    assert_parity(y32.double().cpu().numpy(), ref["y"], f"y f32 (Hq {hq}, Hkv {hkv})")
+    assert bf16_is_rne_of_f32(y, y32)
