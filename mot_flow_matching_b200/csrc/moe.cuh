@@ -192,10 +192,11 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* 
       pos = offsets[e] + blk_base[static_cast<long long>(e) * nblk + t / kMoeRouteTokens] + topk_pos[pr];
       slot[pr] = pos;
     }
-    uint4* dst[kMoeMaxTopK];
+    // the K slot rows (as row numbers: half the registers of pointers)
+    int rowk[kMoeMaxTopK];
 #pragma unroll
-    for (int k = 0; k < kMoeMaxTopK; ++k)
-      dst[k] = reinterpret_cast<uint4*>(xp + static_cast<long long>(__shfl_sync(0xffffffffu, pos, k)) * d);
+    for (int k = 0; k < kMoeMaxTopK; ++k) rowk[k] = __shfl_sync(0xffffffffu, pos, k);
+    uint4* const xp4 = reinterpret_cast<uint4*>(xp);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int c = lane + 32 * i;
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* 
 #pragma unroll
       for (int k = 0; k < kMoeMaxTopK; ++k) {
         if (k >= K) break;
-        dst[k][c] = v[i];
+        xp4[static_cast<long long>(rowk[k]) * n16 + c] = v[i];
       }
     }
     for (int c = lane + 256; c < n16; c += 32) {
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(256) moe_dispatch_kernel(const __nv_bfloat16* 
 #pragma unroll
       for (int k = 0; k < kMoeMaxTopK; ++k) {
         if (k >= K) break;
-        dst[k][c] = w;
+        xp4[static_cast<long long>(rowk[k]) * n16 + c] = w;
       }
     }
   }
