@@ -83,3 +83,22 @@ def test_relabelling_experts_changes_nothing():
         w2[k] = w[k][perm]
     np.testing.assert_allclose(EO.moe_forward(w["x"], w, 3)["y"], EO.moe_forward(w["x"], w2, 3)["y"], rtol=0,
                                atol=1e-12)
+
+
+@pytest.mark.parametrize("E,top_k", [(5, 2), (6, 3), (7, 1)])
+def test_routing_is_the_heaviest_subset_by_brute_force(E, top_k):
+    # over every k-subset of the experts: the routed set is the one with the
+    # largest total probability (probabilities drawn distinct, so it is
+    # unique), and the weights are that subset's probabilities over their sum
+    import itertools
+    g = np.random.default_rng(10 + E)
+    x, wr = g.standard_normal((9, 4)), 2 * g.standard_normal((E, 4))
+    ex, wt, p = EO.route(x, wr, top_k)
+    for t in range(x.shape[0]):
+        best = max(itertools.combinations(range(E), top_k), key=lambda s: sum(p[t, list(s)]))
+        assert set(ex[t]) == set(best)
+        for k, e in enumerate(ex[t]):
+            assert wt[t, k] == pytest.approx(p[t, e] / sum(p[t, list(best)]), rel=1e-13)
+    # the probabilities themselves: softmax written out for one token
+    z = x[0] @ wr.T
+    np.testing.assert_allclose(p[0], np.exp(z) / np.exp(z).sum(), rtol=1e-13)
