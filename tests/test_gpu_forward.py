@@ -226,3 +226,20 @@ def test_fwd_other_head_groupings(cuda_ready, hidden, hq, hkv):
     ref = oracle_forward(wl, t)
     assert_parity(y32.double().cpu().numpy(), ref["y"], f"y f32 (Hq {hq}, Hkv {hkv})")
     assert bf16_is_rne_of_f32(y, y32)
+
+
+def test_fwd_1536x2720_cfg_full(cuda_ready):
+    # the pages' measured end-to-end image size, 1536 x 2720: 48 x 85 patch
+    # tokens = 4080 per branch, not a multiple of the 256-query unit or the
+    # 128-key tile, at the full layer dims with CFG over 400 cached keys
+    # (branch 1 with a 231-token prompt); every output element compared
+    wl = synth.Workload("fwd_1536x2720_cfg2", 2, 4080, 400, 32, 32.0)
+    t = synth.make_inputs(wl, 6100, with_dy=False)
+    t["prefix_len"] = torch.tensor([400, 231], dtype=torch.int32)
+    td = to_dev(t)
+    layer = make_layer(wl, td)
+    y, y32, _, status = run_forward(layer, td)
+    assert status == 0
+    ref = oracle_forward(wl, t)
+    assert_parity(y32.double().cpu().numpy(), ref["y"], "y f32")
+    assert bf16_is_rne_of_f32(y, y32)
